@@ -1,0 +1,421 @@
+"""Benchmark: hybrid block-sparse + linear attention on B200.
+
+One step = one pass of the forward hot path over one synthetic batch:
+sla_build_mask (pool, score, classify) + sla_sparse_attention (critical
+blocks) + sla_linear_combine (marginal blocks, projection, combine).  The
+default workload is the 1.3B-DiT-shaped SLA forward (B=1, H=12, N=32760,
+d=128, bf16, blocks of 64, 5% critical / 10% marginal); ``--workload``
+selects another.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+Multi-GPU (launched by torchrun): every rank runs its own independent problem
+(its own batch element, seed = rank) -- weak scaling, no collective on the
+data path; the only collectives are the timing barrier and the max over
+ranks of the elapsed device time.
+
+``--impl reference`` times the float64 CPU oracle (test infrastructure, the
+reference arm of this benchmark) on the host cores, on a bounded sample of the
+same workload (one head per step), and reports the same metric.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_linear_mean_b200 import synth  # noqa: E402
+
+METRIC = ("hybrid sparse attention ms/call & effective TFLOP/s vs B200 roofline, "
+          "32k–245k")
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+# fp32 FMA peak of a B200 from unit counts and clocks: 148 SMs x 128 FP32
+# lanes x 2 flops x 1.965 GHz (max SM clock).
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes per launch of the dominant kernel from an ncu capture of the
+# current kernel version (None until captured for that version).
+TRAFFIC_PER_LAUNCH = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="sla_1p3b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------- work counts
+
+
+def block_sizes(n, b):
+    return np.array([min((i + 1) * b, n) - i * b for i in range(math.ceil(n / b))],
+                    dtype=np.float64)
+
+
+def effective_flops(wl, mask_np, N=None):
+    """Algorithmic flops of one forward over ``mask_np [B,H,Nqb,Nkb]``:
+    4*d per kept critical (query, key) token pair, plus the linear branch
+    (2*Bk*d^2 + Bk*d per key block for the summaries, |M_i|*(d^2+d) per
+    query block for the gather, 2*d^2 + 2*d per token for phi(q) H / phi(q).z,
+    2*d^2 per token for the projection, tokens of rows with marginal blocks).
+    Real tokens only (ragged tails at their true size)."""
+    N = wl.N if N is None else N
+    d = wl.d
+    sq, sk = block_sizes(N, wl.block_q), block_sizes(N, wl.block_k)
+    crit = (mask_np == 2).astype(np.float64)
+    pairs = float(np.einsum("bhij,i,j->", crit, sq, sk))
+    fl = 4.0 * d * pairs
+    lin = 0.0
+    if wl.frac_marg > 0:
+        marg = (mask_np == 1)
+        nm = marg.sum(axis=-1).astype(np.float64)          # [B,H,Nqb]
+        BH = mask_np.shape[0] * mask_np.shape[1]
+        lin += BH * float(np.sum(2.0 * sk * d * d + sk * d))
+        lin += float(nm.sum()) * (d * d + d)
+        tok = float(np.einsum("bhi,i->", (nm > 0).astype(np.float64), sq))
+        lin += tok * (2.0 * d * d + 2.0 * d + 2.0 * d * d)
+    return fl + lin, pairs, fl, lin
+
+
+# --------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    from block_sparse_linear_mean_b200 import sla
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    x = synth.make_inputs(wl, seed=rank, device=dev)
+    p = sla.params_for(wl)
+    ws_m = sla.workspace(p, sla.SLA_OP_MASK, dev)
+    ws_f = sla.workspace(p, sla.SLA_OP_FORWARD, dev)
+    N, nqb, nkb = wl.N, math.ceil(wl.N / wl.block_q), math.ceil(wl.N / wl.block_k)
+    B, H, d = wl.B, wl.H, wl.d
+    mask = torch.empty(B, H, nqb, nkb, dtype=torch.int8, device=dev)
+    rows = sla.BlockLists.empty(B * H * nqb, nkb, dev)
+    rc = rows.c()
+    out = torch.empty_like(x.q)
+    o_s = torch.empty(x.q.shape, dtype=torch.float32, device=dev)
+    lse = torch.empty(x.q.shape[:-1], dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def chk(name, st):
+        if st != sla.SLA_OK:
+            raise sla.SlaError(name, st)
+
+    def stage_mask(q, k):
+        chk("sla_build_mask", sla.sla_build_mask(p, q.data_ptr(), k.data_ptr(), mask.data_ptr(),
+                                                 rc, None, None, None, ws_m.data_ptr(),
+                                                 ws_m.numel(), sp))
+
+    def stage_sparse(q, k, v):
+        chk("sla_sparse_attention", sla.sla_sparse_attention(
+            p, q.data_ptr(), k.data_ptr(), v.data_ptr(), rc, o_s.data_ptr(), lse.data_ptr(),
+            ws_f.data_ptr(), ws_f.numel(), sp))
+
+    def stage_linear(q, k, v, dst):
+        chk("sla_linear_combine", sla.sla_linear_combine(
+            p, q.data_ptr(), k.data_ptr(), v.data_ptr(), x.proj.data_ptr(), rc,
+            o_s.data_ptr(), dst.data_ptr(), None, ws_f.data_ptr(), ws_f.numel(), sp))
+
+    launches_per_step = 4 + 1 + (2 if wl.frac_marg > 0 else 1)
+
+    # warm-up (also fixes the mask used to count the algorithmic work)
+    for _ in range(max(args.warmup, 0)):
+        stage_mask(x.q, x.k)
+        stage_sparse(x.q, x.k, x.v)
+        stage_linear(x.q, x.k, x.v, out)
+    torch.cuda.synchronize(dev)
+    assert sla.check_device_status(ws_f) == sla.SLA_OK
+    flops, pairs, crit_fl, lin_fl = effective_flops(wl, mask.cpu().numpy())
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        for s in range(args.steps):
+            flush.zero_()                      # L2 flush, outside the timed events
+            e = ev[s]
+            e[0].record(stream)
+            stage_mask(x.q, x.k)
+            e[1].record(stream)
+            stage_sparse(x.q, x.k, x.v)
+            e[2].record(stream)
+            stage_linear(x.q, x.k, x.v, out)
+            e[3].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t_mask = [e[0].elapsed_time(e[1]) for e in ev]
+    t_sparse = [e[1].elapsed_time(e[2]) for e in ev]
+    t_lin = [e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end through the C ABI with host buffers: H2D of q, k, v from
+    # pinned memory, mask + forward, D2H of the output, every step
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (x.q, x.k, x.v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        qd, kd, vd = (torch.empty_like(x.q) for _ in range(3))
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for s in range(args.steps):
+            flush.zero_()
+            ee[s][0].record(stream)
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            stage_mask(qd, kd)
+            stage_sparse(qd, kd, vd)
+            stage_linear(qd, kd, vd, out)
+            oh.copy_(out, non_blocking=True)
+            ee[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(3 * x.q.numel() * x.q.element_size()),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+               "ms_per_step": e2e_ms / args.steps}
+
+    peaks, peak_src = load_peaks()
+    sparse_ms = statistics.mean(t_sparse)
+    tc = _tc_enabled(p)
+    if tc:
+        peak, bound, unit = peaks["bf16_tflops_sustained"], "tensor", "TFLOP/s"
+        peak_note = f"bf16 dense, sustained ({peak_src})"
+    else:
+        peak, bound, unit = FP32_SIMT_PEAK_TFLOPS, "alu", "TFLOP/s"
+        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"
+    achieved = crit_fl / (sparse_ms * 1e-3) / 1e12
+    roofline = {"bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
+                "unit": unit, "frac": round(achieved / peak, 4),
+                "traffic": TRAFFIC_PER_LAUNCH.get((args.workload, "attn_tc" if tc else "attn_simt")),
+                "kernel": "sparse attention forward (" + ("tcgen05" if tc else "SIMT fp32") + ")",
+                "peak_source": peak_note,
+                "algorithmic": f"{crit_fl:.4g} flops per launch = 4*d*{pairs:.4g} kept critical token pairs"}
+    res = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (smooth 3D-grid field + noise, seeded)",
+        "config": {"workload": wl.description, "name": wl.name, "B": B, "H": H, "N": N, "d": d,
+                   "block_q": wl.block_q, "block_k": wl.block_k, "mode": wl.mode,
+                   "frac_crit": wl.frac_crit, "frac_marg": wl.frac_marg, "thr": wl.thr,
+                   "parallelism": f"independent problem per GPU x{world}",
+                   "l2": "256 MB write flushes L2 between steps, outside the timed events"},
+        "breakdown_ms": {"mask": round(statistics.mean(t_mask), 4),
+                         "sparse_attention": round(sparse_ms, 4),
+                         "linear_combine": round(statistics.mean(t_lin), 4)},
+        "work": {"effective_flops_per_step": flops, "critical_flops": crit_fl,
+                 "linear_flops": lin_fl, "critical_token_pairs": pairs,
+                 "kept_fraction_of_dense_pairs": pairs / (B * H * float(N) * N)},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    return res
+
+
+def _tc_enabled(p):
+    """Whether the forward of ``p`` runs the tcgen05 kernel (library query)."""
+    from block_sparse_linear_mean_b200 import sla
+    return sla.sla_forward_uses_tensor_cores(p) == 1
+
+
+# --------------------------------------------------------------- oracle arms
+
+
+def oracle_sample(wl, heads, min_seconds=0.0):
+    """Time the float64 oracle (mask + forward) head by head on the host."""
+    from oracle import sla_oracle as orc
+    x = synth.make_inputs(wl, seed=0, device="cpu", heads=heads)
+    done, flops, t0 = 0, 0.0, time.perf_counter()
+    while done < heads:
+        h = done
+        qh, kh, vh = (t[:, h:h + 1] for t in (x.q, x.k, x.v))
+        m = orc.build_mask(qh, kh, wl.block_q, wl.block_k, wl.mode, wl.frac_crit,
+                           wl.frac_marg, wl.thr)
+        orc.forward(qh, kh, vh, x.proj, m["mask"], wl.block_q, wl.block_k)
+        flops += effective_flops(wl, m["mask"])[0]
+        done += 1
+        if time.perf_counter() - t0 >= min_seconds and min_seconds > 0:
+            break
+    return done, flops, time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl):
+    heads, flops, secs = oracle_sample(wl, heads=min(wl.H, 4), min_seconds=10.0)
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"float64 oracle mask + forward on {heads} of {wl.H} heads "
+                      f"({secs:.1f} s); value = effective flops of those heads / time",
+            "ms_per_call_extrapolated": round(secs / heads * wl.H * 1e3, 1)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample(wl, heads=1)
+    tot_f, tot_s = 0.0, 0.0
+    for _ in range(args.steps):
+        _, f, s = oracle_sample(wl, heads=1)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    cores = blas_threads()
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_s / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": wl.description, "name": wl.name,
+                   "sample": "one head per step (mask + forward) of the workload"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "kind": "oracle",
+                         "cores": cores,
+                         "sample": "float64 oracle, one head per step, host cores"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res))
+        return
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            wl = synth.WORKLOADS[args.workload]
+            if not args.no_cpu_baseline and world == 1:
+                res["cpu_baseline"] = cpu_baseline(wl)
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

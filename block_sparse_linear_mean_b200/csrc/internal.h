@@ -1,0 +1,89 @@
+// Internal launch interface of libsla (host side, not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sla.h"
+
+namespace sla {
+
+using i64 = int64_t;
+
+// Everything a launcher needs about one problem, derived from sla_params.
+struct Geom {
+  int B, H, N, d;
+  int bq, bk;          // block sizes
+  int nqb, nkb;        // block counts
+  int BH;              // B * H
+  int dtype;           // sla_dtype
+  int mode;            // sla_mask_mode
+  int n_c, n_m;        // top-k counts (n_m also used in CDF mode)
+  uint64_t thr_fx;     // ceil(thr * 2^62): CDF threshold in 2^-62 fixed point
+  double thr;
+  float scale;
+  int flags;
+  bool linear;         // linear branch on (frac_marg > 0)
+};
+
+constexpr double kFixedOne = 4611686018427387904.0;  // 2^62
+constexpr float kTieEps = 1e-5f;
+constexpr int kMaxBlocks = 8192;                     // Nqb, Nkb limit
+
+// mask path
+cudaError_t launch_pool(const void* x, int dtype, float* out, int BH, int N,
+                        int d, int block, cudaStream_t s);
+cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
+                          const Geom& g, cudaStream_t s);
+cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
+                            const sla_block_lists& rows, float* scores,
+                            int32_t* tie_count, cudaStream_t s);
+cudaError_t launch_rows_from_mask(const int8_t* mask, const Geom& g,
+                                  const sla_block_lists& rows, cudaStream_t s);
+cudaError_t launch_cols_from_mask(const int8_t* mask, const Geom& g,
+                                  const sla_block_lists& cols, cudaStream_t s);
+
+// forward
+cudaError_t launch_attn_simt(const void* q, const void* k, const void* v,
+                             const Geom& g, const sla_block_lists& rows,
+                             float* o_s, float* lse, cudaStream_t s);
+bool attn_tc_supported(const Geom& g);
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v,
+                           const Geom& g, const sla_block_lists& rows,
+                           float* o_s, float* lse, int32_t* status,
+                           void* scratch, cudaStream_t s);
+size_t attn_tc_scratch_bytes(const Geom& g);
+cudaError_t launch_lin_summary(const void* k, const void* v, const Geom& g,
+                               float* hsum, float* zsum, cudaStream_t s);
+cudaError_t launch_lin_apply(const void* q, const float* hsum,
+                             const float* zsum, const sla_block_lists& rows,
+                             const float* o_s, const float* proj, void* out,
+                             float* o_lin, const Geom& g, cudaStream_t s);
+
+// backward
+cudaError_t launch_bwd_prep(const void* dout, const float* o_s,
+                            const float* o_lin, const float* proj,
+                            float* delta, float* gbuf, float* dw_part,
+                            const Geom& g, cudaStream_t s);
+cudaError_t launch_bwd_dw_reduce(const float* dw_part, float* dproj,
+                                 const Geom& g, cudaStream_t s);
+cudaError_t launch_attn_bwd_dq(const void* q, const void* k, const void* v,
+                               const void* dout, const float* lse,
+                               const float* delta, const sla_block_lists& rows,
+                               float* dq, const Geom& g, cudaStream_t s);
+cudaError_t launch_attn_bwd_dkdv(const void* q, const void* k, const void* v,
+                                 const void* dout, const float* lse,
+                                 const float* delta,
+                                 const sla_block_lists& cols, float* dk,
+                                 float* dv, const Geom& g, cudaStream_t s);
+cudaError_t launch_lin_bwd_q(const void* q, const float* hsum,
+                             const float* zsum, const sla_block_lists& rows,
+                             const float* gbuf, const float* o_lin, float* dq,
+                             float* dhm, float* dzm, const Geom& g,
+                             cudaStream_t s);
+cudaError_t launch_lin_bwd_kv(const void* k, const void* v, const float* dhm,
+                              const float* dzm, const sla_block_lists& cols,
+                              float* dk, float* dv, const Geom& g,
+                              cudaStream_t s);
+
+}  // namespace sla

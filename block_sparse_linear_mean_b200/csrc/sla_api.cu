@@ -1,0 +1,336 @@
+// C ABI of libsla: argument validation, workspace layout and kernel
+// dispatch.  Every entry point only enqueues work on the caller's stream.
+#include <math.h>
+#include <string.h>
+
+#include "internal.h"
+
+namespace sla {
+int bwd_dw_parts(const Geom& g);
+}
+
+using sla::Geom;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int count_from_fraction(double f, int nkb) {
+  double c = ceil(f * static_cast<double>(nkb) - 1e-9);
+  if (c < 0) c = 0;
+  if (c > nkb) c = nkb;
+  return static_cast<int>(c);
+}
+
+sla_status make_geom(const sla_params* p, Geom* g) {
+  if (!p) return SLA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->N < 1 || p->d < 1 || p->block_q < 1 || p->block_k < 1)
+    return SLA_ERR_INVALID_ARG;
+  if (p->dtype != SLA_F32 && p->dtype != SLA_BF16) return SLA_ERR_INVALID_ARG;
+  if (p->mask_mode != SLA_MASK_TOPK && p->mask_mode != SLA_MASK_CDF) return SLA_ERR_INVALID_ARG;
+  if (!(p->frac_crit >= 0.0 && p->frac_crit <= 1.0)) return SLA_ERR_INVALID_ARG;
+  if (!(p->frac_marg >= 0.0 && p->frac_marg <= 1.0)) return SLA_ERR_INVALID_ARG;
+  if (p->mask_mode == SLA_MASK_TOPK && p->frac_crit + p->frac_marg > 1.0 + 1e-9)
+    return SLA_ERR_INVALID_ARG;
+  if (p->mask_mode == SLA_MASK_CDF && !(p->thr >= 0.0 && p->thr < 1.0)) return SLA_ERR_INVALID_ARG;
+  if (!(p->scale >= 0.0f) || !isfinite(p->scale)) return SLA_ERR_INVALID_ARG;
+  if (p->flags & ~SLA_FLAG_SIMT) return SLA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
+  if ((p->block_q != 64 && p->block_q != 128) || (p->block_k != 64 && p->block_k != 128))
+    return SLA_ERR_UNSUPPORTED;
+  g->B = p->B; g->H = p->H; g->N = p->N; g->d = p->d;
+  g->bq = p->block_q; g->bk = p->block_k;
+  g->nqb = (p->N + p->block_q - 1) / p->block_q;
+  g->nkb = (p->N + p->block_k - 1) / p->block_k;
+  if (g->nqb > sla::kMaxBlocks || g->nkb > sla::kMaxBlocks) return SLA_ERR_UNSUPPORTED;
+  const int64_t bh = static_cast<int64_t>(p->B) * p->H;
+  if (bh > 65535) return SLA_ERR_UNSUPPORTED;  // grid y/z dimension limit
+  if (bh * g->nqb >= (int64_t(1) << 31) || bh * g->nkb >= (int64_t(1) << 31) ||
+      bh * p->N >= (int64_t(1) << 31))
+    return SLA_ERR_UNSUPPORTED;
+  g->BH = static_cast<int>(bh);
+  g->dtype = p->dtype;
+  g->mode = p->mask_mode;
+  g->n_c = p->mask_mode == SLA_MASK_TOPK ? count_from_fraction(p->frac_crit, g->nkb) : 0;
+  g->n_m = count_from_fraction(p->frac_marg, g->nkb);
+  if (p->mask_mode == SLA_MASK_TOPK && g->n_m > g->nkb - g->n_c) g->n_m = g->nkb - g->n_c;
+  g->thr = p->thr;
+  g->thr_fx = static_cast<uint64_t>(ceil(p->thr * sla::kFixedOne));
+  g->scale = p->scale > 0.0f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  g->flags = p->flags;
+  g->linear = p->frac_marg > 0.0;
+  return SLA_OK;
+}
+
+bool has_linear_branch(const Geom& g) { return g.linear; }
+
+
+// Workspace layouts (each region 256-byte aligned).
+struct MaskWs { size_t qbar, kbar, logits, total; };
+struct FwdWs { size_t o_s, hsum, zsum, tc, total; };
+struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, total; };
+
+MaskWs mask_ws(const Geom& g) {
+  MaskWs w;
+  size_t off = kStatusBytes;
+  w.qbar = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d);
+  w.kbar = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+  w.logits = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.nkb);
+  w.total = off;
+  return w;
+}
+
+FwdWs fwd_ws(const Geom& g) {
+  FwdWs w;
+  size_t off = kStatusBytes;
+  w.o_s = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.N * g.d);
+  w.hsum = w.zsum = off;
+  if (has_linear_branch(g)) {
+    w.hsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d * g.d);
+    w.zsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+  }
+  w.tc = off; off = align_up(off + sla::attn_tc_scratch_bytes(g));
+  w.total = off;
+  return w;
+}
+
+BwdWs bwd_ws(const Geom& g) {
+  BwdWs w;
+  size_t off = kStatusBytes;
+  w.delta = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.N);
+  w.gbuf = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.N * g.d);
+  w.hsum = w.zsum = w.dhm = w.dzm = off;
+  if (has_linear_branch(g)) {
+    w.hsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d * g.d);
+    w.zsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+    w.dhm = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d * g.d);
+    w.dzm = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d);
+  }
+  w.dwp = off; off = align_up(off + sizeof(float) * size_t(sla::bwd_dw_parts(g)) * g.d * g.d);
+  w.total = off;
+  return w;
+}
+
+bool lists_ok(const sla_block_lists* l) {
+  return l && l->crit_cnt && l->crit_idx && l->marg_cnt && l->marg_idx &&
+         aligned16(l->crit_cnt) && aligned16(l->crit_idx) && aligned16(l->marg_cnt) &&
+         aligned16(l->marg_idx);
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+#define SLA_CUDA(call)                              \
+  do {                                              \
+    if ((call) != cudaSuccess) return SLA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int32_t sla_abi_version(void) { return SLA_ABI_VERSION; }
+
+const char* sla_status_string(sla_status s) {
+  switch (s) {
+    case SLA_OK: return "ok";
+    case SLA_ERR_INVALID_ARG: return "invalid argument";
+    case SLA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SLA_ERR_WORKSPACE: return "workspace too small";
+    case SLA_ERR_CUDA: return "CUDA runtime error";
+    case SLA_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+sla_status sla_validate(const sla_params* p) {
+  Geom g;
+  return make_geom(p, &g);
+}
+
+sla_status sla_workspace_size(const sla_params* p, int32_t op, size_t* bytes) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!bytes) return SLA_ERR_INVALID_ARG;
+  switch (op) {
+    case SLA_OP_MASK: *bytes = mask_ws(g).total; return SLA_OK;
+    case SLA_OP_FORWARD: *bytes = fwd_ws(g).total; return SLA_OK;
+    case SLA_OP_BACKWARD: *bytes = bwd_ws(g).total; return SLA_OK;
+  }
+  return SLA_ERR_INVALID_ARG;
+}
+
+sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
+                          int8_t* mask, const sla_block_lists* rows,
+                          const sla_block_lists* cols, float* scores,
+                          int32_t* tie_count, void* ws, size_t ws_bytes,
+                          void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!q || !k || !mask || !ws || !aligned16(q) || !aligned16(k) || !aligned16(mask) ||
+      !aligned16(ws) || !lists_ok(rows) || (cols && !lists_ok(cols)) ||
+      (scores && !aligned16(scores)) ||
+      (tie_count && (reinterpret_cast<uintptr_t>(tie_count) & 3u)))
+    return SLA_ERR_INVALID_ARG;
+  const MaskWs w = mask_ws(g);
+  if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
+  float* qbar = at<float>(ws, w.qbar);
+  float* kbar = at<float>(ws, w.kbar);
+  float* logits = at<float>(ws, w.logits);
+  SLA_CUDA(sla::launch_pool(q, g.dtype, qbar, g.BH, g.N, g.d, g.bq, s));
+  SLA_CUDA(sla::launch_pool(k, g.dtype, kbar, g.BH, g.N, g.d, g.bk, s));
+  SLA_CUDA(sla::launch_logits(qbar, kbar, logits, g, s));
+  SLA_CUDA(sla::launch_classify(logits, g, mask, *rows, scores, tie_count, s));
+  if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
+  return SLA_OK;
+}
+
+sla_status sla_mask_lists(const sla_params* p, const int8_t* mask,
+                          const sla_block_lists* rows,
+                          const sla_block_lists* cols, void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!mask || (!rows && !cols) || (rows && !lists_ok(rows)) || (cols && !lists_ok(cols)))
+    return SLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rows) SLA_CUDA(sla::launch_rows_from_mask(mask, g, *rows, s));
+  if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
+  return SLA_OK;
+}
+
+static bool tensor_ok(const void* x) { return x && aligned16(x); }
+
+sla_status sla_sparse_attention(const sla_params* p, const void* q, const void* k,
+                                const void* v, const sla_block_lists* rows,
+                                float* o_s, float* lse, void* ws, size_t ws_bytes,
+                                void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o_s) ||
+      !tensor_ok(lse) || !tensor_ok(ws) || !lists_ok(rows))
+    return SLA_ERR_INVALID_ARG;
+  const FwdWs w = fwd_ws(g);
+  if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
+  const bool tc = g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g);
+  if (tc)
+    SLA_CUDA(sla::launch_attn_tc(q, k, v, g, *rows, o_s, lse, at<int32_t>(ws, 0),
+                                 at<void>(ws, w.tc), s));
+  else
+    SLA_CUDA(sla::launch_attn_simt(q, k, v, g, *rows, o_s, lse, s));
+  return SLA_OK;
+}
+
+sla_status sla_linear_combine(const sla_params* p, const void* q, const void* k,
+                              const void* v, const float* proj,
+                              const sla_block_lists* rows, const float* o_s,
+                              void* out, float* o_lin, void* ws, size_t ws_bytes,
+                              void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(proj) ||
+      !tensor_ok(o_s) || !tensor_ok(out) || !tensor_ok(ws) || !lists_ok(rows) ||
+      (o_lin && !aligned16(o_lin)))
+    return SLA_ERR_INVALID_ARG;
+  const FwdWs w = fwd_ws(g);
+  if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* hsum = nullptr;
+  float* zsum = nullptr;
+  if (has_linear_branch(g)) {
+    hsum = at<float>(ws, w.hsum);
+    zsum = at<float>(ws, w.zsum);
+    SLA_CUDA(sla::launch_lin_summary(k, v, g, hsum, zsum, s));
+  }
+  SLA_CUDA(sla::launch_lin_apply(q, hsum, zsum, *rows, o_s, proj, out, o_lin, g, s));
+  return SLA_OK;
+}
+
+sla_status sla_forward(const sla_params* p, const void* q, const void* k,
+                       const void* v, const float* proj,
+                       const sla_block_lists* rows, void* out, float* lse,
+                       float* o_s, float* o_lin, void* ws, size_t ws_bytes,
+                       void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(proj) ||
+      !tensor_ok(out) || !tensor_ok(lse) || !tensor_ok(ws) || !lists_ok(rows) ||
+      (o_s && !aligned16(o_s)) || (o_lin && !aligned16(o_lin)))
+    return SLA_ERR_INVALID_ARG;
+  const FwdWs w = fwd_ws(g);
+  if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  float* os = o_s ? o_s : at<float>(ws, w.o_s);
+  st = sla_sparse_attention(p, q, k, v, rows, os, lse, ws, ws_bytes, stream);
+  if (st != SLA_OK) return st;
+  return sla_linear_combine(p, q, k, v, proj, rows, os, out, o_lin, ws, ws_bytes, stream);
+}
+
+sla_status sla_backward(const sla_params* p, const void* q, const void* k,
+                        const void* v, const float* proj, const void* dout,
+                        const sla_block_lists* rows,
+                        const sla_block_lists* cols, const float* o_s,
+                        const float* lse, const float* o_lin, float* dq,
+                        float* dk, float* dv, float* dproj, void* ws,
+                        size_t ws_bytes, void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  const void* ptrs[] = {q, k, v, proj, dout, o_s, lse, o_lin, dq, dk, dv, dproj, ws};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return SLA_ERR_INVALID_ARG;
+  if (!lists_ok(rows) || !lists_ok(cols)) return SLA_ERR_INVALID_ARG;
+  const BwdWs w = bwd_ws(g);
+  if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
+  float* delta = at<float>(ws, w.delta);
+  float* gbuf = at<float>(ws, w.gbuf);
+  float* dwp = at<float>(ws, w.dwp);
+  SLA_CUDA(sla::launch_bwd_prep(dout, o_s, o_lin, proj, delta, gbuf, dwp, g, s));
+  SLA_CUDA(sla::launch_attn_bwd_dq(q, k, v, dout, lse, delta, *rows, dq, g, s));
+  SLA_CUDA(sla::launch_attn_bwd_dkdv(q, k, v, dout, lse, delta, *cols, dk, dv, g, s));
+  if (has_linear_branch(g)) {
+    float* hsum = at<float>(ws, w.hsum);
+    float* zsum = at<float>(ws, w.zsum);
+    float* dhm = at<float>(ws, w.dhm);
+    float* dzm = at<float>(ws, w.dzm);
+    SLA_CUDA(sla::launch_lin_summary(k, v, g, hsum, zsum, s));
+    SLA_CUDA(sla::launch_lin_bwd_q(q, hsum, zsum, *rows, gbuf, o_lin, dq, dhm, dzm, g, s));
+    SLA_CUDA(sla::launch_lin_bwd_kv(k, v, dhm, dzm, *cols, dk, dv, g, s));
+  }
+  SLA_CUDA(sla::launch_bwd_dw_reduce(dwp, dproj, g, s));
+  return SLA_OK;
+}
+
+int32_t sla_forward_uses_tensor_cores(const sla_params* p) {
+  Geom g;
+  if (make_geom(p, &g) != SLA_OK) return -1;
+  return (g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g)) ? 1 : 0;
+}
+
+sla_status sla_check_device_status(void* ws, void* stream) {
+  if (!ws) return SLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+  int32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  return word == 0 ? SLA_OK : static_cast<sla_status>(word);
+}
+
+}  // extern "C"

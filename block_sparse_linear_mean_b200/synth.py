@@ -31,6 +31,7 @@ implementations.
 
 from __future__ import annotations
 
+import functools
 import math
 from dataclasses import dataclass, field, replace
 from typing import Optional, Tuple
@@ -112,8 +113,10 @@ def reflect_index(i: int, n: int) -> int:
     return i if i < n else period - 1 - i
 
 
+@functools.lru_cache(maxsize=None)
 def gaussian_operator(n: int, sigma: float, truncate: float = 4.0) -> torch.Tensor:
-    """Dense ``(n, n)`` matrix applying a truncated Gaussian blur along one axis."""
+    """Dense ``(n, n)`` matrix applying a truncated Gaussian blur along one axis
+    (cached; callers copy it with ``.to``)."""
     radius = int(truncate * sigma + 0.5)
     offs = torch.arange(-radius, radius + 1, dtype=torch.float64)
     w = torch.exp(-0.5 * (offs / sigma) ** 2)
@@ -138,7 +141,7 @@ def smooth_field(grid, d: int, sigma: float, gen: torch.Generator,
     x = torch.einsum("ct,frtd->frcd", mc, x)
     x = x.reshape(f * r * c, d)
     x = x - x.mean(dim=0, keepdim=True)
-    x = x / x.std(dim=0, keepdim=True).clamp_min(1e-12)
+    x = x / x.std(dim=0, keepdim=True, correction=0).clamp_min(1e-12)
     return x
 
 

@@ -159,16 +159,14 @@ def classify_cdf_row(p_row, thr: float, n_m: int = 0) -> Tuple[np.ndarray, float
     nkb = p_row.shape[0]
     order = rank_order(p_row)
     ps = p_row[order]
-    tail = 0.0
-    kept = nkb
-    tails = np.empty(nkb + 1)
-    tails[nkb] = 0.0
-    for r in range(nkb - 1, 0, -1):          # the top rank is never dropped
-        if tail + ps[r] < thr:
-            tail += ps[r]
-            kept = r
-        else:
-            break
+    # Running tail sums of the walk: tails[r] = ps[r] + ps[r+1] + ... summed
+    # from the lowest rank upward (np.cumsum adds in exactly that order).  The
+    # tail sums never decrease as r falls, so "drop while the tail including
+    # the block stays below thr" drops exactly the ranks with tails[r] < thr;
+    # the top rank is never dropped.
+    tails = np.cumsum(ps[::-1])[::-1]
+    kept = max(1, int(np.count_nonzero(tails >= thr)))
+    tail = float(tails[kept]) if kept < nkb else 0.0
     # tail sums at the two ranks that decide the cut
     t_kept_last = tail + ps[kept - 1]        # tail sum including last kept
     # at thr <= 0 no tail sum can fall below thr, so no decision is close
@@ -315,6 +313,42 @@ def linear_attention_rows(q_rows, hsum, zsum, marg_blocks):
     zm = zsum[marg_blocks].sum(axis=0)
     f = phi(q_rows)
     return (f @ hm) / (f @ zm)[:, None]
+
+
+def linear_summaries_of(k, v, blocks, block_k: int):
+    """Summaries of the listed key blocks only (one head): ``{j: (H_j, z_j)}``."""
+    k, v = f64(k), f64(v)
+    n = k.shape[0]
+    out = {}
+    for j in blocks:
+        a, b = block_range(int(j), n, block_k)
+        pk = phi(k[a:b])
+        out[int(j)] = (pk.T @ v[a:b], pk.sum(axis=0))
+    return out
+
+
+def forward_rows(q, k, v, proj, mask_row, block_i: int, block_q: int,
+                 block_k: int, scale: Optional[float] = None) -> Dict:
+    """a4-a7 for the tokens of one query block of one head (``q, k, v``:
+    ``[N, d]``), from that block's mask row.  Used to check sampled rows of
+    workloads too large for the whole oracle."""
+    q = f64(q)
+    n, d = q.shape
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    a, e = block_range(block_i, n, block_q)
+    mask_row = np.asarray(mask_row)
+    crit = np.nonzero(mask_row == CRITICAL)[0]
+    marg = np.nonzero(mask_row == MARGINAL)[0]
+    o_s, lse = sparse_attention_rows(q[a:e], k, v, crit, block_k, s)
+    if len(marg):
+        summ = linear_summaries_of(k, v, marg, block_k)
+        hm = sum(summ[int(j)][0] for j in marg)
+        zm = sum(summ[int(j)][1] for j in marg)
+        f = phi(q[a:e])
+        o_lin = (f @ hm) / (f @ zm)[:, None]
+    else:
+        o_lin = np.zeros_like(q[a:e])
+    return dict(out=o_s + o_lin @ f64(proj), o_s=o_s, lse=lse, o_lin=o_lin)
 
 
 def linear_attention(q, k, v, mask, block_q: int, block_k: int):
