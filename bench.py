@@ -25,7 +25,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -53,7 +52,7 @@ TRAFFIC_PER_LAUNCH = {}
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="sla_1p3b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -107,58 +106,70 @@ def effective_flops(wl, mask_np, N=None):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and clock-event (throttle) reasons of one GPU every
+    20 ms through NVML in a background thread while the timed region runs;
+    raw samples go to gpurun_out/clocks_rank<i>.csv."""
 
-    def __init__(self, device_index):
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+               "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+    def __init__(self, device_index, period_s=0.02):
         self.idx = device_index
-        self.proc = None
+        self.period = period_s
+        self.samples = []
+        self.err = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
 
+    def _run(self):
+        import pynvml as nv
+        h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((time.time(), sm, rs, pw))
+            except Exception as e:  # keep sampling; record the last error
+                self.err = repr(e)
+            self._stop.wait(self.period)
+
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self.thread = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        except Exception as e:
+            self.err = repr(e)
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.fh.close()
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            with open(self.path, "w") as f:
+                f.write("t,sm_mhz,reasons_mask,power_w\n")
+                for t, sm, rs, pw in self.samples:
+                    f.write(f"{t:.3f},{sm},{rs:#x},{pw:.1f}\n")
+        except OSError:
+            pass
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for name, val in zip(names, parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": [f"no samples ({self.err})"]}
+        reasons = sorted({name for _, _, rs, _ in self.samples
+                          for name, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(sm for _, sm, _, _ in self.samples),
+                "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": reasons,
+                "samples": len(self.samples),
+                "power_w_max": max(pw for _, _, _, pw in self.samples)}
 
 
 # --------------------------------------------------------------- our arm

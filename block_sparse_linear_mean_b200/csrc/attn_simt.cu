@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const i64 head = i64(bh) * N * D;
   const int list_row = bh * nqb + qb;
-  const int ncrit = rows.crit_cnt[list_row];
+  const int ncrit = min(max(rows.crit_cnt[list_row], 0), nkb);
   const int32_t* crit = rows.crit_idx + i64(list_row) * nkb;
 
   // stage the CTA's query rows (zero beyond N)

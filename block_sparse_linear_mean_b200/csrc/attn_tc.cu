@@ -1,14 +1,610 @@
-// Tensor-core (tcgen05) block-sparse attention forward: not built yet; the
-// SIMT kernel serves every configuration until it is.
-#include "internal.h"
+// Block-sparse exact attention forward on the 5th-generation tensor cores
+// (tcgen05 + TMEM + TMA), bf16 inputs, fp32 accumulation.
+//
+// SLA post ("Selective Linear Attention", list "the idea"): critical blocks go
+// through FlashAttention -- exact online-softmax attention -- and negligible
+// blocks are skipped.  NABLA post point 4: compute only on the kept blocks.
+//
+// Work decomposition
+//   * A CTA owns a 128-row query tile of one (batch, head): one query block
+//     of 128 rows, or two consecutive query blocks of 64 rows.  A small plan
+//     kernel merges the tile's critical lists into one ascending list of key
+//     blocks with a membership bit per query block; key tiles are 128 keys
+//     (one block of 128 or two listed blocks of 64).  A row only attends to
+//     keys whose block is in its own query block's list (masked otherwise).
+//   * Warp 0 (one lane): TMA producer -- Q once, then K and V per key tile
+//     into a 2-stage ring, with the 3D tensor map [B*H, N, d] so rows past N
+//     read as zeros.
+//   * Warp 1 (one lane): MMA issuer -- S = Q K^T (M=128, N=128, K=d) into a
+//     double-buffered TMEM tile, O += P V (M=128, N=d, K=128) into TMEM.
+//   * Warps 2-5: one thread per query row -- tcgen05.ld of its S row, masking,
+//     online softmax in the exp2 domain with lazy rescaling (the running max
+//     is only moved when it grows by more than 2^8, which keeps P <= 256),
+//     P as bf16 into a 128B-swizzled shared-memory tile, and the epilogue
+//     O / l and LSE.
+// Every mbarrier wait is bounded: on expiry the CTA records SLA_ERR_TIMEOUT
+// in the status word, drains, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
 
 namespace sla {
 
-bool attn_tc_supported(const Geom&) { return false; }
-size_t attn_tc_scratch_bytes(const Geom&) { return 0; }
-cudaError_t launch_attn_tc(const void*, const void*, const void*, const Geom&,
-                           const sla_block_lists&, float*, float*, int32_t*,
-                           void*, cudaStream_t) {
+namespace {
+
+constexpr int kTileM = 128;
+constexpr int kTileN = 128;
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
+// columns [col, col+32) of TMEM lane (lane_base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  uint32_t r[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Values produced by tcgen05.ld may only be read after tcgen05.wait::ld; this
+// empty asm (ordered after the wait) re-defines them so no use of a loaded
+// value can be scheduled above the wait.
+template <int K>
+__device__ __forceinline__ void reg_fence(float* v) {
+#pragma unroll
+  for (int i = 0; i < K; ++i) asm volatile("" : "+f"(v[i]));
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
+// 1; addresses and byte offsets are encoded in 16-byte units.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator,
+// A/B K-major (0) or MN-major (1), N >> 3 at bit 17, M >> 4 at bit 24.
+constexpr uint32_t idesc_bf16(int m, int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ plan
+// One key-tile descriptor packs two 16-bit entries (the second only used for
+// key blocks of 64): bit 15 present, bits 13-14 membership (bit 13: query
+// block of rows 0-63, bit 14: rows 64-127; both for a 128-row block), bits
+// 0-12 key-block index.
+
+constexpr uint32_t kPresent = 1u << 15;
+
+__device__ __forceinline__ uint32_t entry(int blk, uint32_t flags) {
+  return kPresent | (flags << 13) | static_cast<uint32_t>(blk);
+}
+
+__global__ void plan_kernel(sla_block_lists rows, int BH, int nqb, int nkb, int nqt, int bq,
+                            int bk, int32_t* __restrict__ cnt, uint32_t* __restrict__ tiles) {
+  const int tile = blockIdx.x * blockDim.x + threadIdx.x;
+  if (tile >= BH * nqt) return;
+  const int bh = tile / nqt, qt = tile % nqt;
+  const int qa = bq == 128 ? qt : 2 * qt;
+  const int qb = (bq == 64 && 2 * qt + 1 < nqb) ? 2 * qt + 1 : -1;
+  const uint32_t fa = bq == 128 ? 3u : 1u;
+  const int ra = bh * nqb + qa;
+  const int na = min(max(rows.crit_cnt[ra], 0), nkb);
+  const int32_t* la = rows.crit_idx + i64(ra) * nkb;
+  int nb = 0;
+  const int32_t* lb = nullptr;
+  if (qb >= 0) {
+    const int rb = bh * nqb + qb;
+    nb = min(max(rows.crit_cnt[rb], 0), nkb);
+    lb = rows.crit_idx + i64(rb) * nkb;
+  }
+  uint32_t* out = tiles + i64(tile) * nkb;
+  int ia = 0, ib = 0, nt = 0;
+  uint32_t pending = 0;
+  const int per_tile = kTileN / bk;  // 1 or 2 entries per key tile
+  int in_tile = 0;
+  while (ia < na || ib < nb) {
+    const int a = ia < na ? la[ia] : 0x7fffffff;
+    const int b = ib < nb ? lb[ib] : 0x7fffffff;
+    int blk;
+    uint32_t f;
+    if (a == b) { blk = a; f = fa | 2u; ++ia; ++ib; }
+    else if (a < b) { blk = a; f = fa; ++ia; }
+    else { blk = b; f = 2u; ++ib; }
+    if (blk < 0 || blk >= nkb) continue;  // malformed list entry
+    pending |= entry(blk, f) << (16 * in_tile);
+    if (++in_tile == per_tile) {
+      out[nt++] = pending;
+      pending = 0;
+      in_tile = 0;
+      if (nt == nkb) break;  // only reachable with duplicated list entries
+    }
+  }
+  if (in_tile && nt < nkb) out[nt++] = pending;
+  cnt[tile] = nt;
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int D, int BQ, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ plan_cnt,
+               const uint32_t* __restrict__ plan_tiles, int plan_stride, float* __restrict__ o_s,
+               float* __restrict__ lse, int32_t* status, int N, int nqt, float scale_log2,
+               long long timeout_cycles, int debug_skip) {
+  constexpr int DC = D / 64;                  // 64-element (128 B) chunks along d
+  constexpr uint32_t kQBytes = DC * 16384;    // Q tile 128 x D bf16
+  constexpr uint32_t kKBytes = DC * 16384;    // K tile 128 x D
+  constexpr uint32_t kPBytes = 2 * 16384;     // P tile 128 x 128 bf16
+  constexpr uint32_t offQ = 0;
+  constexpr uint32_t offK = offQ + kQBytes;
+  constexpr uint32_t offV = offK + kStages * kKBytes;
+  constexpr uint32_t offP = offV + kStages * kKBytes;
+  constexpr uint32_t offBar = offP + 2 * kPBytes;
+  constexpr uint32_t kTileBytes = 2 * kKBytes;  // K + V per stage
+  constexpr uint32_t idesc_qk = idesc_bf16(128, kTileN, 0, 0);
+  constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(base);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
+  // barrier indices
+  const uint32_t b_q = smem_u32(&bars[0]);
+  auto b_kv_full = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto b_kv_empty = [&](int s) { return smem_u32(&bars[3 + s]); };
+  auto b_s_full = [&](int b) { return smem_u32(&bars[5 + b]); };
+  auto b_s_free = [&](int b) { return smem_u32(&bars[7 + b]); };
+  auto b_p_full = [&](int b) { return smem_u32(&bars[9 + b]); };
+  auto b_pv_done = [&](int b) { return smem_u32(&bars[11 + b]); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[13]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[14]);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tile = blockIdx.x;
+  const int bh = tile / nqt, qt = tile % nqt;
+  const int T = plan_cnt[tile];
+  const uint32_t* ptiles = plan_tiles + i64(tile) * plan_stride;
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q, 1);
+    for (int s = 0; s < kStages; ++s) { mbar_init(b_kv_full(s), 1); mbar_init(b_kv_empty(s), 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_s_full(b), 1);
+      mbar_init(b_s_free(b), 4);
+      mbar_init(b_p_full(b), 4);
+      mbar_init(b_pv_done(b), 1);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // TMEM: 512 columns (S0 | S1 | O)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO = tmem + 256;
+
+  // bounded wait: false on timeout or when another role gave up
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    const long long t0 = clock64();
+    for (uint32_t it = 0;; ++it) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((it & 255u) == 255u) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > timeout_cycles) {
+          *abort_flag = 1;
+          atomicExch(status, static_cast<int32_t>(SLA_ERR_TIMEOUT));
+          return false;
+        }
+      }
+    }
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0 && T > 0) {
+      mbar_expect_tx(b_q, kQBytes);
+#pragma unroll
+      for (int c = 0; c < DC; ++c) tma_load_3d(sb + offQ + c * 16384, &tmQ, c * 64, qt * kTileM, bh, b_q);
+      for (int t = 0; t < T; ++t) {
+        const int s = t % kStages;
+        if (t >= kStages && !wait(b_kv_empty(s), ((t / kStages) & 1) ^ 1)) break;
+        if (debug_skip && tile == 0 && t == 0) continue;  // test aid: never arrives
+        const uint32_t desc = ptiles[t];
+        mbar_expect_tx(b_kv_full(s), kTileBytes);
+        const uint32_t kdst = sb + offK + s * kKBytes, vdst = sb + offV + s * kKBytes;
+        if (BK == 128) {
+          const int blk = desc & 0x1FFF;
+#pragma unroll
+          for (int c = 0; c < DC; ++c) {
+            tma_load_3d(kdst + c * 16384, &tmK, c * 64, blk * 128, bh, b_kv_full(s));
+            tma_load_3d(vdst + c * 16384, &tmV, c * 64, blk * 128, bh, b_kv_full(s));
+          }
+        } else {
+          const int blk0 = desc & 0x1FFF;
+          const int blk1 = (desc >> 16) & kPresent ? (desc >> 16) & 0x1FFF : blk0;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int blk = e ? blk1 : blk0;
+#pragma unroll
+            for (int c = 0; c < DC; ++c) {
+              tma_load_3d(kdst + c * 16384 + e * 8192, &tmK, c * 64, blk * 64, bh, b_kv_full(s));
+              tma_load_3d(vdst + c * 16384 + e * 8192, &tmV, c * 64, blk * 64, bh, b_kv_full(s));
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && T > 0) {
+      bool ok = wait(b_q, 0);
+      auto issue_s = [&](int t) -> bool {
+        const int s = t % kStages, b = t & 1;
+        if (!wait(b_kv_full(s), (t / kStages) & 1)) return false;
+        if (t >= 2 && !wait(b_s_free(b), ((t >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t kbase = sb + offK + s * kKBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          tc_mma(tS[b], sdesc(sb + offQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), idesc_qk,
+                 kk > 0);
+        }
+        tc_commit(b_s_full(b));
+        return true;
+      };
+      auto issue_pv = [&](int t) -> bool {
+        const int s = t % kStages, b = t & 1;
+        if (!wait(b_p_full(b), (t >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t pbase = sb + offP + b * kPBytes;
+        const uint32_t vbase = sb + offV + s * kKBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk) {
+          const uint32_t poff = (kk / 4) * 16384 + (kk % 4) * 32;
+          tc_mma(tO, sdesc(pbase + poff, 16, 1024), sdesc(vbase + kk * 2048, 16384, 1024),
+                 idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(b_kv_empty(s));
+        tc_commit(b_pv_done(b));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int t = 0; ok && t < T; ++t) {
+        if (t + 1 < T) ok = issue_s(t + 1);
+        if (ok) ok = issue_pv(t);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int quad = warp & 3;            // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;       // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t rflag = BQ == 128 ? 3u : (r < 64 ? 1u : 2u);
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint8_t* prow_base = base + offP + r * 128;
+    for (int t = 0; ok && t < T; ++t) {
+      const int b = t & 1;
+      const uint32_t desc = ptiles[t];
+      if (!__all_sync(0xffffffffu, wait(b_s_full(b), (t >> 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      float s[kTileN];
+#pragma unroll
+      for (int c = 0; c < kTileN; c += 32) tmem_ld32(tS[b] + lane_off + c, s + c);
+      tmem_wait_ld();
+      reg_fence<kTileN>(s);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_s_free(b));
+      // mask and tile max (log2 domain)
+      float mt = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kTileN / BK; ++e) {
+        const uint32_t ent = (desc >> (16 * e)) & 0xFFFFu;
+        const int blk = ent & 0x1FFF;
+        const bool member = (ent & kPresent) && (((ent >> 13) & 3u) & rflag);
+        const int kvalid = member ? min(BK, N - blk * BK) : 0;
+#pragma unroll
+        for (int c = 0; c < BK; ++c) {
+          const float x = c < kvalid ? s[e * BK + c] * scale_log2 : -INFINITY;
+          s[e * BK + c] = x;
+          mt = fmaxf(mt, x);
+        }
+      }
+      // running max with lazy rescale
+      bool rescale = false;
+      float alpha = 1.f;
+      if (mt > -INFINITY) {
+        if (m_ref == -INFINITY) {
+          m_ref = mt;
+        } else if (mt > m_ref + kRescaleLog2) {
+          alpha = exp2f(m_ref - mt);
+          m_ref = mt;
+          l *= alpha;
+          rescale = true;
+        }
+      }
+      float rs = 0.f;
+      uint32_t pk[kTileN / 2];
+#pragma unroll
+      for (int c = 0; c < kTileN; c += 2) {
+        const float p0 = m_ref == -INFINITY ? 0.f : exp2f(s[c] - m_ref);
+        const float p1 = m_ref == -INFINITY ? 0.f : exp2f(s[c + 1] - m_ref);
+        rs += p0 + p1;
+        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+        pk[c / 2] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      l += rs;
+      // P buffer b is free once PV of tile t-2 completed
+      if (t >= 2 && !__all_sync(0xffffffffu, wait(b_pv_done(b), ((t >> 1) & 1) ^ 1))) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = prow_base + b * kPBytes;
+#pragma unroll
+      for (int u = 0; u < kTileN / 8; ++u) {  // 16-byte units of 8 keys
+        const int ch = u / 8, uu = u % 8;
+        uint4 val = make_uint4(pk[u * 4], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
+        *reinterpret_cast<uint4*>(prow + ch * 16384 + ((uu ^ (r & 7)) << 4)) = val;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // rescale O (warp-wide TMEM access) once the previous PV is complete
+      if (__any_sync(0xffffffffu, rescale)) {
+        if (t >= 1 && !__all_sync(0xffffffffu, wait(b_pv_done((t - 1) & 1), ((t - 1) >> 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          tmem_ld32(tO + lane_off + c, o);
+          tmem_wait_ld();
+          reg_fence<32>(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tO + lane_off + c, o);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_p_full(b));
+    }
+    // epilogue: O / l, LSE
+    const int row = qt * kTileM + r;
+    const i64 orow = (i64(bh) * N + row) * D;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    bool fin = ok && T > 0;  // warp-uniform
+    if (fin) fin = __all_sync(0xffffffffu, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
+    if (fin) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        tmem_ld32(tO + lane_off + c, o);
+        tmem_wait_ld();
+        reg_fence<32>(o);
+        if (row < N) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(o_s + orow + c + i) =
+                make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        }
+      }
+    } else if (row < N) {
+      for (int c = 0; c < D; c += 4)
+        *reinterpret_cast<float4*>(o_s + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (row < N)
+      lse[i64(bh) * N + row] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }
+
+  // teardown: on an abort let in-flight copies and MMAs drain (bounded)
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000) { __nanosleep(1000); }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [B*H, N, d] bf16 viewed as a 3D tensor (d fastest); box of 64 x rows x 1
+// with 128-byte swizzle, rows past N read as zeros.
+bool make_map(CUtensorMap* m, const void* ptr, const Geom& g, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.N),
+                        static_cast<cuuint64_t>(g.BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.d) * 2,
+                           static_cast<cuuint64_t>(g.N) * g.d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return static_cast<size_t>(D / 64) * 16384 * (1 + 2 * kStages) + 2 * 32768 + 256 + 1024;
+}
+
+template <int D, int BQ, int BK>
+cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const int32_t* cnt, const uint32_t* tiles, const Geom& g, int nqt, float* o_s,
+                     float* lse, int32_t* status, cudaStream_t s) {
+  auto kern = attn_tc_kernel<D, BQ, BK>;
+  const size_t smem = smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const float scale_log2 = g.scale * 1.4426950408889634f;
+  const bool debug = (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0;
+  const long long timeout = debug ? (1ll << 24) : (1ll << 31);
+  kern<<<g.BH * nqt, kThreads, smem, s>>>(mq, mk, mv, cnt, tiles, g.nkb, o_s, lse, status, g.N,
+                                          nqt, scale_log2, timeout, debug ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_tc_supported(const Geom& g) {
+  return g.dtype == SLA_BF16 && (g.d == 64 || g.d == 128) && (g.bq == 64 || g.bq == 128) &&
+         (g.bk == 64 || g.bk == 128) && encode_fn() != nullptr;
+}
+
+size_t attn_tc_scratch_bytes(const Geom& g) {
+  const size_t nqt = (static_cast<size_t>(g.N) + kTileM - 1) / kTileM;
+  const size_t tiles = static_cast<size_t>(g.BH) * nqt;
+  return tiles * sizeof(int32_t) + 256 + tiles * g.nkb * sizeof(uint32_t);
+}
+
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const Geom& g,
+                           const sla_block_lists& rows, float* o_s, float* lse, int32_t* status,
+                           void* scratch, cudaStream_t s) {
+  const int nqt = (g.N + kTileM - 1) / kTileM;
+  const size_t ntiles = static_cast<size_t>(g.BH) * nqt;
+  int32_t* cnt = static_cast<int32_t*>(scratch);
+  uint32_t* tiles = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) +
+                                                ((ntiles * sizeof(int32_t) + 255) & ~size_t(255)));
+  plan_kernel<<<static_cast<unsigned>((ntiles + 127) / 128), 128, 0, s>>>(
+      rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, cnt, tiles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, g, kTileM) || !make_map(&mk, k, g, g.bk) || !make_map(&mv, v, g, g.bk))
+    return cudaErrorInvalidValue;
+#define SLA_TC_CASE(D_, BQ_, BK_)                                                              \
+  if (g.d == D_ && g.bq == BQ_ && g.bk == BK_)                                                 \
+    return launch_t<D_, BQ_, BK_>(mq, mk, mv, cnt, tiles, g, nqt, o_s, lse, status, s);
+  SLA_TC_CASE(128, 64, 64)
+  SLA_TC_CASE(128, 64, 128)
+  SLA_TC_CASE(128, 128, 64)
+  SLA_TC_CASE(128, 128, 128)
+  SLA_TC_CASE(64, 64, 64)
+  SLA_TC_CASE(64, 64, 128)
+  SLA_TC_CASE(64, 128, 64)
+  SLA_TC_CASE(64, 128, 128)
+#undef SLA_TC_CASE
   return cudaErrorNotSupported;
 }
 

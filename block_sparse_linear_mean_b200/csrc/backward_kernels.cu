@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const i64 head = i64(bh) * N * D;
   const int list_row = bh * nqb + qb;
-  const int ncrit = rows.crit_cnt[list_row];
+  const int ncrit = min(max(rows.crit_cnt[list_row], 0), nkb);
   const int32_t* crit = rows.crit_idx + i64(list_row) * nkb;
   for (int e = threadIdx.x * 4; e < 64 * D; e += 1024) {
     const int r = e / D, c = e % D, t = row0 + r;
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dkdv_kernel(
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const i64 head = i64(bh) * N * D;
   const int col = bh * nkb + kb;
-  const int nq = cols.crit_cnt[col];
+  const int nq = min(max(cols.crit_cnt[col], 0), nqb);
   const int32_t* qlist = cols.crit_idx + i64(col) * nqb;
   for (int e = threadIdx.x * 4; e < 64 * D; e += 1024) {
     const int r = e / D, c = e % D, t = key0 + r;
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(256) lin_bwd_q_kernel(
   float* sc = Q + 8 * D;       // [8] den, [8] dden
   const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int list_row = bh * nqb + i;
-  const int nmarg = rows.marg_cnt[list_row];
+  const int nmarg = min(max(rows.marg_cnt[list_row], 0), nkb);
   if (nmarg == 0) return;
   const int32_t* marg = rows.marg_idx + i64(list_row) * nkb;
   const i64 head = i64(bh) * N * D;
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(256) lin_bwd_kv_kernel(
   float* Vt = Kt + 8 * D;      // [8][D]
   const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int col = bh * nkb + j;
-  const int nq = cols.marg_cnt[col];
+  const int nq = min(max(cols.marg_cnt[col], 0), nqb);
   if (nq == 0) return;
   const int32_t* qlist = cols.marg_idx + i64(col) * nqb;
   const i64 head = i64(bh) * N * D;

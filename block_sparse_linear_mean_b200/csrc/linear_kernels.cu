@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256) lin_apply_kernel(
   const int i = blockIdx.x, bh = blockIdx.y;
   const int list_row = bh * nqb + i;
   // without summaries (linear branch off) marginal entries are ignored
-  const int nmarg = hsum ? rows.marg_cnt[list_row] : 0;
+  const int nmarg = hsum ? min(max(rows.marg_cnt[list_row], 0), nkb) : 0;
   const int32_t* marg = rows.marg_idx + i64(list_row) * nkb;
   const i64 head = i64(bh) * N * D;
   const int t0 = i * bq, t1 = min(t0 + bq, N);

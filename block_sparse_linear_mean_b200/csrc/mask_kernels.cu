@@ -315,21 +315,24 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
   }
   __syncthreads();
 
-  // tie report: the decisive gaps of this row, as seen in fp32 P
+  // tie report: the decisive margins of this row, as seen in fp32 P -- score
+  // gaps at a cut relative to the higher score, tail sums against thr in
+  // absolute (unit mass) terms
   if (a.tie_count && tid == 0) {
     auto pr = [&](int r) { return __uint_as_float(static_cast<uint32_t>(keys[r] >> 32)); };
+    auto close = [&](int r) { return (pr(r) - pr(r + 1)) <= kTieEps * pr(r); };
     bool tie = false;
     if (a.mode == SLA_MASK_TOPK) {
-      if (c > 0 && c < nkb) tie |= (pr(c - 1) - pr(c)) <= kTieEps;
+      if (c > 0 && c < nkb) tie |= close(c - 1);
     } else if (a.thr_fx > 0) {
       const double thr = static_cast<double>(a.thr_fx) / kFixedOne;
       if (c > 1) tie |= fabs(static_cast<double>(t_at[0]) / kFixedOne - thr) <= kTieEps;
       if (c < nkb) {
         tie |= fabs(thr - static_cast<double>(t_at[1]) / kFixedOne) <= kTieEps;
-        tie |= (pr(c - 1) - pr(c)) <= kTieEps;
+        tie |= close(c - 1);
       }
     }
-    if (nm > 0 && c + nm < nkb) tie |= (pr(c + nm - 1) - pr(c + nm)) <= kTieEps;
+    if (nm > 0 && c + nm < nkb) tie |= close(c + nm - 1);
     if (tie) atomicAdd(a.tie_count, 1);
   }
 

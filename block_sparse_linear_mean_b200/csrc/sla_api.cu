@@ -38,7 +38,7 @@ sla_status make_geom(const sla_params* p, Geom* g) {
     return SLA_ERR_INVALID_ARG;
   if (p->mask_mode == SLA_MASK_CDF && !(p->thr >= 0.0 && p->thr < 1.0)) return SLA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0f) || !isfinite(p->scale)) return SLA_ERR_INVALID_ARG;
-  if (p->flags & ~SLA_FLAG_SIMT) return SLA_ERR_INVALID_ARG;
+  if (p->flags & ~(SLA_FLAG_SIMT | SLA_FLAG_DEBUG_TIMEOUT)) return SLA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if ((p->block_q != 64 && p->block_q != 128) || (p->block_k != 64 && p->block_k != 128))
     return SLA_ERR_UNSUPPORTED;

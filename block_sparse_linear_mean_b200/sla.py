@@ -32,6 +32,7 @@ SLA_F32, SLA_BF16 = 0, 1
 SLA_MASK_TOPK, SLA_MASK_CDF = 0, 1
 SLA_OP_MASK, SLA_OP_FORWARD, SLA_OP_BACKWARD = 0, 1, 2
 SLA_FLAG_SIMT = 1
+SLA_FLAG_DEBUG_TIMEOUT = 2
 
 # Entry points declared in include/sla.h (checked by the test-suite).
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",

@@ -100,6 +100,11 @@ typedef struct {
 
 /* Force the portable fp32 SIMT kernels even for bf16 inputs (testing aid). */
 #define SLA_FLAG_SIMT 1
+/* Testing aid for the failure path: the tensor-core attention kernel's first
+ * CTA withholds one K/V tile load and every bounded device-side wait gives up
+ * after ~1e7 cycles instead of ~2e9, so the call ends with SLA_ERR_TIMEOUT in
+ * the status word (read by sla_check_device_status) instead of hanging. */
+#define SLA_FLAG_DEBUG_TIMEOUT 2
 
 /* Compressed block lists.  Row lists (CSR): for each of the B*H*Nqb query
  * blocks r, crit_cnt[r] critical key-block indices in ascending order at
@@ -131,8 +136,9 @@ SLA_API sla_status sla_workspace_size(const sla_params* p, int32_t op, size_t* b
  *   rows       CSR lists out (required)
  *   cols       CSC lists out (nullable)
  *   scores     [B,H,Nqb,Nkb] fp32 out, row-softmaxed pooled scores (nullable)
- *   tie_count  one int32 out: rows whose decisive score gap / tail sum lies
- *              within 1e-5 of the cut (nullable) */
+ *   tie_count  one int32 out (nullable): rows whose selection sits within
+ *              1e-5 of a decision -- a score gap at a cut within 1e-5 of the
+ *              higher score, or (CDF) a decisive tail sum within 1e-5 of thr */
 SLA_API sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
                           int8_t* mask, const sla_block_lists* rows,
                           const sla_block_lists* cols, float* scores,

@@ -129,10 +129,15 @@ def rank_order(p_row: np.ndarray) -> np.ndarray:
     return np.lexsort((idx, -p_row))
 
 
+def _rel_gap(hi: float, lo: float) -> float:
+    """Score gap at a cut, relative to the higher score (0 for equal scores)."""
+    return (hi - lo) / hi if hi > 0 else 0.0
+
+
 def classify_topk_row(p_row, n_c: int, n_m: int) -> Tuple[np.ndarray, float]:
-    """Label one row by ranks; also return the score gap at each cut (the
-    row's tie margin: the smallest gap between the last block in a class and
-    the first block below it)."""
+    """Label one row by ranks; also return the row's tie margin: the smallest
+    score gap at a cut (last block of a class vs the first block below it),
+    relative to the higher of the two scores."""
     p_row = f64(p_row)
     nkb = p_row.shape[0]
     order = rank_order(p_row)
@@ -143,7 +148,7 @@ def classify_topk_row(p_row, n_c: int, n_m: int) -> Tuple[np.ndarray, float]:
     margin = math.inf
     for cut in (n_c, n_c + n_m):
         if 0 < cut < nkb and not (cut == n_c + n_m and n_m == 0):
-            margin = min(margin, ps[cut - 1] - ps[cut])
+            margin = min(margin, _rel_gap(ps[cut - 1], ps[cut]))
     return labels, margin
 
 
@@ -153,8 +158,9 @@ def classify_cdf_row(p_row, thr: float, n_m: int = 0) -> Tuple[np.ndarray, float
 
     Walk from the lowest rank upward; a block is dropped while the tail sum
     including it is strictly below ``thr``.  Returns labels and the row's
-    margin: the distance of the two decisive tail sums from ``thr`` and the
-    score gap at the cut(s)."""
+    margin: the smaller of the distances of the two decisive tail sums from
+    ``thr`` (absolute, on the unit mass scale) and the score gaps at the cut(s)
+    (relative to the higher score)."""
     p_row = f64(p_row)
     nkb = p_row.shape[0]
     order = rank_order(p_row)
@@ -172,13 +178,13 @@ def classify_cdf_row(p_row, thr: float, n_m: int = 0) -> Tuple[np.ndarray, float
     # at thr <= 0 no tail sum can fall below thr, so no decision is close
     margin = abs(t_kept_last - thr) if (kept > 1 and thr > 0) else math.inf
     if kept < nkb:
-        margin = min(margin, abs(thr - tail), ps[kept - 1] - ps[kept])
+        margin = min(margin, abs(thr - tail), _rel_gap(ps[kept - 1], ps[kept]))
     labels = np.zeros(nkb, dtype=np.int8)
     labels[order[:kept]] = CRITICAL
     n_m = min(n_m, nkb - kept)
     labels[order[kept:kept + n_m]] = MARGINAL
     if n_m > 0 and kept + n_m < nkb:
-        margin = min(margin, ps[kept + n_m - 1] - ps[kept + n_m])
+        margin = min(margin, _rel_gap(ps[kept + n_m - 1], ps[kept + n_m]))
     return labels, margin
 
 

@@ -106,7 +106,8 @@ def test_forward_matches_oracle_with_oracle_mask(case, simt):
     o = orc.forward(x.q, x.k, x.v, x.proj, ref["mask"], wl.block_q, wl.block_k)
     res = {}
     for key in ("o_s", "o_lin", "out"):
-        res[key] = assert_close(to_np(f[key]), o[key], wl.dtype, f"{name}.{key}")
+        res[key] = assert_close(to_np(f[key]), o[key], wl.dtype, f"{name}.{key}",
+                                stored_bf16=(key == "out"))
     lse = to_np(f["lse"])
     fin = np.isfinite(o["lse"])
     np.testing.assert_array_equal(np.isfinite(lse), fin)
@@ -149,7 +150,7 @@ def test_all_critical_equals_dense_attention(dtype):
     x, f, g = _run_with_mask(wl, mask)
     ref = torch.nn.functional.scaled_dot_product_attention(
         x.q.double(), x.k.double(), x.v.double()).numpy()
-    assert_close(to_np(f["out"]), ref, dtype, "dense")
+    assert_close(to_np(f["out"]), ref, dtype, "dense", stored_bf16=True)
 
 
 def test_all_negligible_gives_zero_and_neg_inf():
@@ -196,3 +197,13 @@ def test_device_status_ok_after_calls():
     m = sla.build_mask(p, t["q"], t["k"])
     f = sla.forward(p, t["q"], t["k"], t["v"], t["proj"], m["rows"])
     assert sla.check_device_status(f["ws"]) == sla.SLA_OK
+
+
+def test_bf16_forward_runs_tensor_core_kernel():
+    for name in ("sla_1p3b", "nabla_14b", "long_clip"):
+        p = sla.params_for(synth.WORKLOADS[name])
+        assert sla.sla_forward_uses_tensor_cores(p) == 1, name
+    p = sla.params_for(synth.WORKLOADS["tiny"])
+    assert sla.sla_forward_uses_tensor_cores(p) == 0        # fp32 mode: SIMT
+    p = sla.params_for(synth.WORKLOADS["sla_1p3b"], simt=True)
+    assert sla.sla_forward_uses_tensor_cores(p) == 0
