@@ -21,7 +21,8 @@
 //     online softmax in the exp2 domain with lazy rescaling (the running max
 //     is only moved when it grows by more than 2^8, which keeps P <= 256),
 //     P as bf16 into a 128B-swizzled shared-memory tile, and the epilogue
-//     O / l and LSE.
+//     O / l and LSE.  The row sum l accumulates the bf16-rounded P, the same
+//     weights the PV product uses.
 // Every mbarrier wait is bounded: on expiry the CTA records SLA_ERR_TIMEOUT
 // in the status word, drains, frees its TMEM and returns.
 #include <cuda.h>
@@ -429,9 +430,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int c = 0; c < kTileN; c += 2) {
         const float p0 = m_ref == -INFINITY ? 0.f : exp2f(s[c] - m_ref);
         const float p1 = m_ref == -INFINITY ? 0.f : exp2f(s[c + 1] - m_ref);
-        rs += p0 + p1;
         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
         pk[c / 2] = *reinterpret_cast<uint32_t*>(&h);
+        // the row sum uses the rounded weights the MMA sees, so O / l is an
+        // exact convex combination of V rows
+        const float2 hr = __bfloat1622float2(h);
+        rs += hr.x + hr.y;
       }
       l += rs;
       // P buffer b is free once PV of tile t-2 completed

@@ -37,7 +37,7 @@ cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
                           const Geom& g, cudaStream_t s);
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
                             const sla_block_lists& rows, float* scores,
-                            int32_t* tie_count, cudaStream_t s);
+                            int32_t* tie_count, cudaStream_t s, bool from_prob = false);
 cudaError_t launch_rows_from_mask(const int8_t* mask, const Geom& g,
                                   const sla_block_lists& rows, cudaStream_t s);
 cudaError_t launch_cols_from_mask(const int8_t* mask, const Geom& g,

@@ -207,6 +207,7 @@ __device__ void compact_row(const int8_t* lab, int n, int32_t* idx_c,
 
 struct ClassifyArgs {
   int nkb, S, mode, n_c, n_m;
+  int from_prob;  // input rows are already softmaxed scores, not logits
   uint64_t thr_fx;
   int8_t* mask;
   sla_block_lists rows;
@@ -231,18 +232,22 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
   const int nkb = a.nkb, S = a.S, tid = threadIdx.x;
   const float* lr = logits + i64(row) * nkb;
 
-  // 1. softmax over the row
-  float m = -FLT_MAX;
-  for (int j = tid; j < nkb; j += kCT) m = fmaxf(m, lr[j]);
-  m = block_reduce_max(m, redf);
-  float se = 0.f;
-  for (int j = tid; j < nkb; j += kCT) se += expf(lr[j] - m);
-  se = block_reduce_sum(se, redf);
-  const float inv = 1.0f / se;
+  // 1. softmax over the row (skipped for rows given as scores)
+  float m = 0.f, inv = 1.f;
+  if (!a.from_prob) {
+    m = -FLT_MAX;
+    for (int j = tid; j < nkb; j += kCT) m = fmaxf(m, lr[j]);
+    m = block_reduce_max(m, redf);
+    float se = 0.f;
+    for (int j = tid; j < nkb; j += kCT) se += expf(lr[j] - m);
+    se = block_reduce_sum(se, redf);
+    inv = 1.0f / se;
+  }
   for (int j = tid; j < S; j += kCT) {
     uint64_t key = 0;
     if (j < nkb) {
-      const float p = expf(lr[j] - m) * inv;
+      // scores are non-negative, so their bit patterns order like the values
+      const float p = a.from_prob ? fmaxf(lr[j], 0.f) : expf(lr[j] - m) * inv;
       if (a.scores) a.scores[i64(row) * nkb + j] = p;
       key = (static_cast<uint64_t>(__float_as_uint(p)) << 32) |
             static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(j));
@@ -351,8 +356,9 @@ static int sort_size(int n) {
 
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
                             const sla_block_lists& rows, float* scores,
-                            int32_t* tie_count, cudaStream_t s) {
+                            int32_t* tie_count, cudaStream_t s, bool from_prob) {
   ClassifyArgs a;
+  a.from_prob = from_prob ? 1 : 0;
   a.nkb = g.nkb;
   a.S = sort_size(g.nkb);
   a.mode = g.mode;

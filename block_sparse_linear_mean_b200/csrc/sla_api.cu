@@ -195,6 +195,22 @@ sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
   return SLA_OK;
 }
 
+sla_status sla_classify_scores(const sla_params* p, const float* scores,
+                               int8_t* mask, const sla_block_lists* rows,
+                               const sla_block_lists* cols, int32_t* tie_count,
+                               void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!scores || !mask || !aligned16(scores) || !aligned16(mask) || !lists_ok(rows) ||
+      (cols && !lists_ok(cols)) || (tie_count && (reinterpret_cast<uintptr_t>(tie_count) & 3u)))
+    return SLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(sla::launch_classify(scores, g, mask, *rows, nullptr, tie_count, s, true));
+  if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
+  return SLA_OK;
+}
+
 sla_status sla_mask_lists(const sla_params* p, const int8_t* mask,
                           const sla_block_lists* rows,
                           const sla_block_lists* cols, void* stream) {

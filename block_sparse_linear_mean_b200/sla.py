@@ -36,7 +36,8 @@ SLA_FLAG_DEBUG_TIMEOUT = 2
 
 # Entry points declared in include/sla.h (checked by the test-suite).
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",
-           "sla_workspace_size", "sla_build_mask", "sla_mask_lists",
+           "sla_workspace_size", "sla_build_mask", "sla_classify_scores",
+           "sla_mask_lists",
            "sla_forward", "sla_sparse_attention", "sla_linear_combine",
            "sla_backward", "sla_forward_uses_tensor_cores",
            "sla_check_device_status")
@@ -84,6 +85,9 @@ def lib():
         L.sla_build_mask.restype = ctypes.c_int
         L.sla_build_mask.argtypes = [P(sla_params), VP, VP, VP, P(sla_block_lists),
                                      P(sla_block_lists), VP, VP, VP, SZ, VP]
+        L.sla_classify_scores.restype = ctypes.c_int
+        L.sla_classify_scores.argtypes = [P(sla_params), VP, VP, P(sla_block_lists),
+                                          P(sla_block_lists), VP, VP]
         L.sla_mask_lists.restype = ctypes.c_int
         L.sla_mask_lists.argtypes = [P(sla_params), VP, P(sla_block_lists),
                                      P(sla_block_lists), VP]
@@ -138,6 +142,12 @@ def sla_build_mask(p, q, k, mask, rows, cols, scores, tie_count, ws, ws_bytes, s
     return lib().sla_build_mask(ctypes.byref(p), q, k, mask, ctypes.byref(rows),
                                 ctypes.byref(cols) if cols is not None else None,
                                 scores, tie_count, ws, ws_bytes, stream)
+
+
+def sla_classify_scores(p, scores, mask, rows, cols, tie_count, stream) -> int:
+    return lib().sla_classify_scores(ctypes.byref(p), scores, mask, ctypes.byref(rows),
+                                     ctypes.byref(cols) if cols is not None else None,
+                                     tie_count, stream)
 
 
 def sla_mask_lists(p, mask, rows, cols, stream) -> int:
@@ -257,6 +267,20 @@ def build_mask(p: sla_params, q: torch.Tensor, k: torch.Tensor, want_scores=Fals
                                             rc, cc, _ptr(scores), ties.data_ptr(),
                                             ws.data_ptr(), ws.numel(), _stream()))
     return dict(mask=mask, rows=rows, cols=cols, scores=scores, ties=ties[:1])
+
+
+def classify_scores(p: sla_params, scores: torch.Tensor, want_cols=False) -> dict:
+    """Classify given row-softmaxed pooled scores ``[B,H,Nqb,Nkb]`` fp32."""
+    dev = scores.device
+    B, H, nqb, nkb = scores.shape
+    mask = torch.empty(B, H, nqb, nkb, dtype=torch.int8, device=dev)
+    rows = BlockLists.empty(B * H * nqb, nkb, dev)
+    cols = BlockLists.empty(B * H * nkb, nqb, dev) if want_cols else None
+    ties = torch.zeros(4, dtype=torch.int32, device=dev)
+    _check("sla_classify_scores", sla_classify_scores(
+        p, scores.data_ptr(), mask.data_ptr(), rows.c(), cols.c() if cols else None,
+        ties.data_ptr(), _stream()))
+    return dict(mask=mask, rows=rows, cols=cols, ties=ties[:1])
 
 
 def mask_lists(p: sla_params, mask: torch.Tensor, want_rows=True, want_cols=True):

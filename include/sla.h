@@ -145,6 +145,15 @@ SLA_API sla_status sla_build_mask(const sla_params* p, const void* q, const void
                           int32_t* tie_count, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* Step 3 alone: classify given pooled scores.
+ *   scores     [B,H,Nqb,Nkb] fp32 in: each row a softmax over key blocks
+ *              (non-negative; the selection rule of p is applied as is)
+ *   mask, rows, cols, tie_count as for sla_build_mask.  No workspace. */
+SLA_API sla_status sla_classify_scores(const sla_params* p, const float* scores,
+                               int8_t* mask, const sla_block_lists* rows,
+                               const sla_block_lists* cols, int32_t* tie_count,
+                               void* stream);
+
 /* Row (CSR) and/or column (CSC) lists from any block mask (e.g. one made
  * elsewhere).  Either list pointer may be NULL, not both.  No workspace. */
 SLA_API sla_status sla_mask_lists(const sla_params* p, const int8_t* mask,

@@ -25,15 +25,15 @@ def errors(got, ref):
     return float(e.max()) if e.size else 0.0, float(e.mean()) if e.size else 0.0
 
 
-# Round-to-nearest-even to bf16 moves a value by at most 2^-9 of its
-# magnitude (half a unit in the last of 8 significant bits).
-BF16_HALF_ULP_REL = 2.0 ** -9
+# Round-to-nearest-even to bf16 moves a value by at most half a unit in the
+# last of its 8 significant bits: 2^-8 of the value at the bottom of a binade.
+BF16_HALF_ULP_REL = 2.0 ** -8
 
 
 def assert_close(got, ref, dtype, what, rel=False, stored_bf16=False):
     """Tolerances of the workload statement.  ``stored_bf16``: the value is
     an output stored in bf16, so each element may additionally carry its own
-    output rounding (<= 2^-9 |ref|) on top of the computation's error."""
+    output rounding (<= 2^-8 |ref|) on top of the computation's error."""
     ref = np.asarray(ref, dtype=np.float64)
     got = np.asarray(got, dtype=np.float64)
     scale = max(1e-30, float(np.abs(ref).max())) if rel else 1.0

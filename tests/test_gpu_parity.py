@@ -64,22 +64,26 @@ def test_mask_matches_oracle(case):
     assert lists_from_gpu(got["cols"], ncols, mask.shape[2]) == expected_cols(mask)
 
 
-def test_classifier_alone_is_exact_on_gpu_scores(case):
-    # Given the same fp32 scores, the classification is a pure function of
-    # them: top-k must agree bit for bit; the CDF decision may differ only
-    # where a tail sum lies within 1e-12 of thr.
+def test_classifier_alone_is_exact_on_given_scores(case):
+    # The oracle's scores, rounded once to fp32, are classified by the GPU
+    # (sla_classify_scores) and by the oracle on the very same fp32 values:
+    # top-k must agree bit for bit; the CDF decision may differ only where a
+    # tail sum lies within 1e-12 of thr.
     name, wl, x, t, ref = case
     p = sla.params_from(t["q"], wl)
-    got = sla.build_mask(p, t["q"], t["k"], want_scores=True)
+    s32 = ref["scores"].astype(np.float32)
+    got = sla.classify_scores(p, torch.from_numpy(s32).cuda(), want_cols=True)
     torch.cuda.synchronize()
-    scores = got["scores"].cpu().numpy().astype(np.float64)
-    mask_ref, margins = orc.classify(scores, wl.mode, wl.frac_crit, wl.frac_marg, wl.thr)
+    mask_ref, margins = orc.classify(s32.astype(np.float64), wl.mode, wl.frac_crit,
+                                     wl.frac_marg, wl.thr)
     mask = got["mask"].cpu().numpy()
     if wl.mode == "topk":
         np.testing.assert_array_equal(mask, mask_ref)
     else:
         diff = (mask != mask_ref).any(axis=-1)
         assert not (diff & (margins > 1e-12)).any()
+    ncols = mask.shape[0] * mask.shape[1] * mask.shape[3]
+    assert lists_from_gpu(got["cols"], ncols, mask.shape[2]) == expected_cols(mask)
 
 
 def test_mask_lists_from_oracle_mask(case):
