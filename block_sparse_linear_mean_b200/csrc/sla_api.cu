@@ -350,3 +350,62 @@ sla_status sla_check_device_status(void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of sla_sparse_attention.
+//
+// Its scratch (the attention plan, and the status word when the caller gives
+// none) lives in one file-scope device array of kNoAllocBytes.  Host code
+// only ever sees a host-side stand-in for the array's name, so the device
+// address is looked up once per device, with that device current, by the
+// first call on it, and cached.
+
+#include <mutex>
+
+namespace {
+constexpr size_t kNoAllocBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+extern "C" sla_status sla_sparse_attention_noalloc(const sla_params* p, const void* q,
+                                                   const void* k, const void* v,
+                                                   const sla_block_lists* rows, float* o_s,
+                                                   float* lse, int32_t* status,
+                                                   void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o_s) || !tensor_ok(lse) ||
+      !lists_ok(rows) || (status && (reinterpret_cast<uintptr_t>(status) & 3u)))
+    return SLA_ERR_INVALID_ARG;
+  const bool tc = g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g);
+  const size_t need = kStatusBytes + (tc ? align_up(sla::attn_tc_scratch_bytes(g)) : 0);
+  if (need > kNoAllocBytes) return SLA_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SLA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SLA_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr)
+        return SLA_ERR_CUDA;
+      g_noalloc_addr[dev] = addr;
+    }
+    base = g_noalloc_addr[dev];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* word = status ? status : static_cast<int32_t*>(base);
+  SLA_CUDA(cudaMemsetAsync(word, 0, sizeof(int32_t), s));  // the only state that must start at 0
+  if (tc)
+    SLA_CUDA(sla::launch_attn_tc(q, k, v, g, *rows, o_s, lse, word,
+                                 static_cast<char*>(base) + kStatusBytes, s));
+  else
+    SLA_CUDA(sla::launch_attn_simt(q, k, v, g, *rows, o_s, lse, s));
+  return SLA_OK;
+}

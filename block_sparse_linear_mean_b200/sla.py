@@ -38,7 +38,8 @@ SLA_FLAG_DEBUG_TIMEOUT = 2
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",
            "sla_workspace_size", "sla_build_mask", "sla_classify_scores",
            "sla_mask_lists",
-           "sla_forward", "sla_sparse_attention", "sla_linear_combine",
+           "sla_forward", "sla_sparse_attention", "sla_sparse_attention_noalloc",
+           "sla_linear_combine",
            "sla_backward", "sla_forward_uses_tensor_cores",
            "sla_check_device_status")
 
@@ -97,6 +98,9 @@ def lib():
         L.sla_sparse_attention.restype = ctypes.c_int
         L.sla_sparse_attention.argtypes = [P(sla_params), VP, VP, VP, P(sla_block_lists),
                                            VP, VP, VP, SZ, VP]
+        L.sla_sparse_attention_noalloc.restype = ctypes.c_int
+        L.sla_sparse_attention_noalloc.argtypes = [P(sla_params), VP, VP, VP,
+                                                   P(sla_block_lists), VP, VP, VP, VP]
         L.sla_linear_combine.restype = ctypes.c_int
         L.sla_linear_combine.argtypes = [P(sla_params), VP, VP, VP, VP, P(sla_block_lists),
                                          VP, VP, VP, VP, SZ, VP]
@@ -164,6 +168,12 @@ def sla_forward(p, q, k, v, proj, rows, out, lse, o_s, o_lin, ws, ws_bytes, stre
 def sla_sparse_attention(p, q, k, v, rows, o_s, lse, ws, ws_bytes, stream) -> int:
     return lib().sla_sparse_attention(ctypes.byref(p), q, k, v, ctypes.byref(rows), o_s,
                                       lse, ws, ws_bytes, stream)
+
+
+def sla_sparse_attention_noalloc(p, q, k, v, rows, o_s, lse, status, stream) -> int:
+    """Workspace-free sparse attention (scratch in a static device array)."""
+    return lib().sla_sparse_attention_noalloc(ctypes.byref(p), q, k, v, ctypes.byref(rows),
+                                              o_s, lse, status, stream)
 
 
 def sla_linear_combine(p, q, k, v, proj, rows, o_s, out, o_lin, ws, ws_bytes, stream) -> int:

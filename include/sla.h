@@ -188,6 +188,36 @@ SLA_API sla_status sla_sparse_attention(const sla_params* p, const void* q, cons
                                 float* o_s, float* lse, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* Step 4, critical part, for callers that cannot allocate device memory.
+ * (The pages have no counterpart; this is a deployment variant of
+ * sla_sparse_attention with the same arguments minus the workspace.)
+ *
+ * Some callers get only a stream and their input and output buffers at the
+ * point where they run the attention: plugins of inference runtimes that
+ * hand no allocator or workspace to their enqueue step, and real-time loops
+ * that must not allocate because cudaMalloc synchronises the device and can
+ * fail under memory pressure.  This entry point allocates nothing and calls
+ * no allocating routine.  Its scratch -- the per-query-tile key-block plan of
+ * the tensor-core kernel -- lives in one 16 MiB static device array that
+ * every GPU which loads the library holds until the process exits.
+ *   q, k, v, rows, o_s, lse  as for sla_sparse_attention
+ *   status     one int32 device word (nullable): cleared, then set to
+ *              SLA_ERR_TIMEOUT if a bounded device-side wait gave up; read
+ *              it after synchronising the stream
+ * Returns SLA_ERR_WORKSPACE when the problem needs more than the 16 MiB
+ * (bf16 path: about 4 bytes per (128-row query tile, key block) pair,
+ * B*H*ceil(N/128)*Nkb*4 bytes; the 1.3B-DiT shape needs 6.3 MB, the
+ * 14B-DiT and long-clip shapes are refused).
+ * The first call on each device looks up the array's device address (a
+ * one-time set-up per device); make that first call before any stream
+ * capture.  All calls share the array and it keeps the last call's
+ * contents: calls that may overlap on the GPU (other streams, other host
+ * threads) race with each other and must be serialised by the caller. */
+SLA_API sla_status sla_sparse_attention_noalloc(const sla_params* p, const void* q,
+                                        const void* k, const void* v,
+                                        const sla_block_lists* rows, float* o_s,
+                                        float* lse, int32_t* status, void* stream);
+
 /* Step 4, marginal part and combine: per-key-block summaries, linear
  * attention over each query block's marginal list, out = o_s + O_lin @ proj.
  *   o_s        [B,H,N,d] fp32 in (from sla_sparse_attention)
