@@ -38,7 +38,9 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;                 // two warpgroups
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softmax
+constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -143,6 +145,14 @@ __device__ __forceinline__ void reg_fence(float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 2^x with the hardware approximation (ex2.approx, flush-to-zero): relative
+// error ~2^-22, far below the bf16 rounding P goes through next.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
 // 1; addresses and byte offsets are encoded in 16-byte units.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -225,32 +235,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                float* __restrict__ lse, int32_t* status, int N, int nqt, float scale_log2,
                long long timeout_cycles, int debug_skip) {
   constexpr int DC = D / 64;                  // 64-element (128 B) chunks along d
+  constexpr int DH = D / 2;                   // O columns per softmax half
   constexpr uint32_t kQBytes = DC * 16384;    // Q tile 128 x D bf16
-  constexpr uint32_t kKBytes = DC * 16384;    // K tile 128 x D
+  constexpr uint32_t kKBytes = DC * 16384;    // K (or V) tile 128 x D
   constexpr uint32_t kPBytes = 2 * 16384;     // P tile 128 x 128 bf16
   constexpr uint32_t offQ = 0;
   constexpr uint32_t offK = offQ + kQBytes;
   constexpr uint32_t offV = offK + kStages * kKBytes;
   constexpr uint32_t offP = offV + kStages * kKBytes;
-  constexpr uint32_t offBar = offP + 2 * kPBytes;
-  constexpr uint32_t kTileBytes = 2 * kKBytes;  // K + V per stage
+  constexpr uint32_t offRed = offP + 2 * kPBytes;      // [2 parity][2 halves][128] fp32
+  constexpr uint32_t offBar = offRed + 2 * 2 * 128 * 4;
+  constexpr uint32_t kUsed = offBar + 256;
   constexpr uint32_t idesc_qk = idesc_bf16(128, kTileN, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(base);
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  uint8_t* base = smem_raw + pad;
+  const uint32_t sb = raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
-  // barrier indices
   const uint32_t b_q = smem_u32(&bars[0]);
-  auto b_kv_full = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto b_kv_empty = [&](int s) { return smem_u32(&bars[3 + s]); };
-  auto b_s_full = [&](int b) { return smem_u32(&bars[5 + b]); };
-  auto b_s_free = [&](int b) { return smem_u32(&bars[7 + b]); };
-  auto b_p_full = [&](int b) { return smem_u32(&bars[9 + b]); };
-  auto b_pv_done = [&](int b) { return smem_u32(&bars[11 + b]); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[13]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[14]);
+  auto b_k_full = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto b_v_full = [&](int s) { return smem_u32(&bars[3 + s]); };
+  auto b_k_empty = [&](int s) { return smem_u32(&bars[5 + s]); };
+  auto b_v_empty = [&](int s) { return smem_u32(&bars[7 + s]); };
+  auto b_s_full = [&](int b) { return smem_u32(&bars[9 + b]); };
+  auto b_s_free = [&](int b) { return smem_u32(&bars[11 + b]); };
+  auto b_p_full = [&](int b) { return smem_u32(&bars[13 + b]); };
+  auto b_pv_done = [&](int b) { return smem_u32(&bars[15 + b]); };
+  auto b_red = [&](int b) { return smem_u32(&bars[17 + b]); };
+  const uint32_t b_fin = smem_u32(&bars[19]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[20]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[21]);
+  float* red = reinterpret_cast<float*>(base + offRed);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int tile = blockIdx.x;
@@ -258,15 +276,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int T = plan_cnt[tile];
   const uint32_t* ptiles = plan_tiles + i64(tile) * plan_stride;
 
+  // The dynamic window must hold the 1024-aligned layout; it does whenever
+  // the window starts 1024-aligned (then pad == 0).  Refuse otherwise.
+  if (pad + kUsed > kSmemRequest) {
+    if (threadIdx.x == 0) atomicExch(status, static_cast<int32_t>(SLA_ERR_UNSUPPORTED));
+    return;
+  }
+
   if (threadIdx.x == 0) {
     mbar_init(b_q, 1);
-    for (int s = 0; s < kStages; ++s) { mbar_init(b_kv_full(s), 1); mbar_init(b_kv_empty(s), 1); }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(b_k_full(s), 1);
+      mbar_init(b_v_full(s), 1);
+      mbar_init(b_k_empty(s), 1);
+      mbar_init(b_v_empty(s), 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_s_full(b), 1);
-      mbar_init(b_s_free(b), 4);
-      mbar_init(b_p_full(b), 4);
+      mbar_init(b_s_free(b), kSoftmaxWarps);
+      mbar_init(b_p_full(b), kSoftmaxWarps);
       mbar_init(b_pv_done(b), 1);
+      mbar_init(b_red(b), kSoftmaxWarps);
     }
+    mbar_init(b_fin, kSoftmaxWarps);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -282,6 +314,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO = tmem + 256;
 
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    atomicExch(status, static_cast<int32_t>(SLA_ERR_TIMEOUT));
+  };
   // bounded wait: false on timeout or when another role gave up
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
     const long long t0 = clock64();
@@ -289,47 +325,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (mbar_try_wait(bar, parity)) return true;
       if ((it & 255u) == 255u) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > timeout_cycles) {
-          *abort_flag = 1;
-          atomicExch(status, static_cast<int32_t>(SLA_ERR_TIMEOUT));
-          return false;
-        }
+        if (clock64() - t0 > timeout_cycles) { give_up(); return false; }
       }
     }
   };
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
+    // K of tile t+2 may load once S of tile t has been computed; V of tile
+    // t+2 once P V of tile t has: the two rings advance independently.
     if (lane == 0 && T > 0) {
       mbar_expect_tx(b_q, kQBytes);
 #pragma unroll
       for (int c = 0; c < DC; ++c) tma_load_3d(sb + offQ + c * 16384, &tmQ, c * 64, qt * kTileM, bh, b_q);
-      for (int t = 0; t < T; ++t) {
-        const int s = t % kStages;
-        if (t >= kStages && !wait(b_kv_empty(s), ((t / kStages) & 1) ^ 1)) break;
-        if (debug_skip && tile == 0 && t == 0) continue;  // test aid: never arrives
-        const uint32_t desc = ptiles[t];
-        mbar_expect_tx(b_kv_full(s), kTileBytes);
-        const uint32_t kdst = sb + offK + s * kKBytes, vdst = sb + offV + s * kKBytes;
+      auto load = [&](const CUtensorMap* map, uint32_t dst0, uint32_t bar, uint32_t desc) {
+        mbar_expect_tx(bar, kKBytes);
         if (BK == 128) {
           const int blk = desc & 0x1FFF;
 #pragma unroll
-          for (int c = 0; c < DC; ++c) {
-            tma_load_3d(kdst + c * 16384, &tmK, c * 64, blk * 128, bh, b_kv_full(s));
-            tma_load_3d(vdst + c * 16384, &tmV, c * 64, blk * 128, bh, b_kv_full(s));
-          }
+          for (int c = 0; c < DC; ++c) tma_load_3d(dst0 + c * 16384, map, c * 64, blk * 128, bh, bar);
         } else {
           const int blk0 = desc & 0x1FFF;
-          const int blk1 = (desc >> 16) & kPresent ? (desc >> 16) & 0x1FFF : blk0;
+          const int blk1 = ((desc >> 16) & kPresent) ? (desc >> 16) & 0x1FFF : blk0;
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int blk = e ? blk1 : blk0;
+          for (int e = 0; e < 2; ++e)
 #pragma unroll
-            for (int c = 0; c < DC; ++c) {
-              tma_load_3d(kdst + c * 16384 + e * 8192, &tmK, c * 64, blk * 64, bh, b_kv_full(s));
-              tma_load_3d(vdst + c * 16384 + e * 8192, &tmV, c * 64, blk * 64, bh, b_kv_full(s));
-            }
-          }
+            for (int c = 0; c < DC; ++c)
+              tma_load_3d(dst0 + c * 16384 + e * 8192, map, c * 64, (e ? blk1 : blk0) * 64, bh, bar);
+        }
+      };
+      int tk = 0, tv = 0;
+      long long t0 = clock64();
+      while (tv < T) {
+        bool moved = false;
+        if (tk < T && (tk < kStages || mbar_try_wait(b_k_empty(tk % kStages), ((tk / kStages) & 1) ^ 1))) {
+          if (!(debug_skip && tile == 0 && tk == 0))  // test aid: tile 0's K never arrives
+            load(&tmK, sb + offK + (tk % kStages) * kKBytes, b_k_full(tk % kStages), ptiles[tk]);
+          ++tk;
+          moved = true;
+        }
+        if (tv < tk && (tv < kStages || mbar_try_wait(b_v_empty(tv % kStages), ((tv / kStages) & 1) ^ 1))) {
+          load(&tmV, sb + offV + (tv % kStages) * kKBytes, b_v_full(tv % kStages), ptiles[tv]);
+          ++tv;
+          moved = true;
+        }
+        if (moved) {
+          t0 = clock64();
+        } else {
+          if (*abort_flag) break;
+          if (clock64() - t0 > timeout_cycles) { give_up(); break; }
         }
       }
     }
@@ -339,7 +383,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = wait(b_q, 0);
       auto issue_s = [&](int t) -> bool {
         const int s = t % kStages, b = t & 1;
-        if (!wait(b_kv_full(s), (t / kStages) & 1)) return false;
+        if (!wait(b_k_full(s), (t / kStages) & 1)) return false;
         if (t >= 2 && !wait(b_s_free(b), ((t >> 1) & 1) ^ 1)) return false;
         tc_fence_after();
         const uint32_t kbase = sb + offK + s * kKBytes;
@@ -350,11 +394,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                  kk > 0);
         }
         tc_commit(b_s_full(b));
+        tc_commit(b_k_empty(s));
         return true;
       };
       auto issue_pv = [&](int t) -> bool {
         const int s = t % kStages, b = t & 1;
         if (!wait(b_p_full(b), (t >> 1) & 1)) return false;
+        if (!wait(b_v_full(s), (t / kStages) & 1)) return false;
         tc_fence_after();
         const uint32_t pbase = sb + offP + b * kPBytes;
         const uint32_t vbase = sb + offV + s * kKBytes;
@@ -364,7 +410,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc_mma(tO, sdesc(pbase + poff, 16, 1024), sdesc(vbase + kk * 2048, 16384, 1024),
                  idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(b_kv_empty(s));
+        tc_commit(b_v_empty(s));
         tc_commit(b_pv_done(b));
         return true;
       };
@@ -376,45 +422,58 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else {
     // ---------------------------------------------------------- softmax
+    // Two warpgroups; thread (h, r) owns columns [64h, 64h + 64) of query
+    // row r and O columns [h*D/2, (h+1)*D/2).  The two halves of a row
+    // exchange their partial maxima through shared memory every tile, so
+    // both keep the same running max and rescale decisions.
+    const int h = (warp - 2) >> 2;        // column half
     const int quad = warp & 3;            // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;       // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t rflag = BQ == 128 ? 3u : (r < 64 ? 1u : 2u);
+    const unsigned full = 0xffffffffu;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow_base = base + offP + r * 128;
+    uint8_t* prow_base = base + offP + h * 16384 + r * 128;
     for (int t = 0; ok && t < T; ++t) {
       const int b = t & 1;
       const uint32_t desc = ptiles[t];
-      if (!__all_sync(0xffffffffu, wait(b_s_full(b), (t >> 1) & 1))) { ok = false; break; }
+      // this thread's 64 keys: entry h of a tile of two 64-blocks, or half h
+      // of one 128-block
+      const uint32_t ent = BK == 64 ? (desc >> (16 * h)) & 0xFFFFu : desc & 0xFFFFu;
+      const int blk = ent & 0x1FFF;
+      const bool member = (ent & kPresent) && (((ent >> 13) & 3u) & rflag);
+      const int kvalid = member ? max(0, min(64, N - blk * BK - (BK == 128 ? h * 64 : 0))) : 0;
+      if (!__all_sync(full, wait(b_s_full(b), (t >> 1) & 1))) { ok = false; break; }
       tc_fence_after();
-      float s[kTileN];
-#pragma unroll
-      for (int c = 0; c < kTileN; c += 32) tmem_ld32(tS[b] + lane_off + c, s + c);
+      float s[64];
+      tmem_ld32(tS[b] + lane_off + h * 64, s);
+      tmem_ld32(tS[b] + lane_off + h * 64 + 32, s + 32);
       tmem_wait_ld();
-      reg_fence<kTileN>(s);
+      reg_fence<64>(s);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_s_free(b));
-      // mask and tile max (log2 domain)
-      float mt = -INFINITY;
+      // partial max of the raw scores over this thread's valid keys
+      float mx = -INFINITY;
+      if (kvalid == 64) {
 #pragma unroll
-      for (int e = 0; e < kTileN / BK; ++e) {
-        const uint32_t ent = (desc >> (16 * e)) & 0xFFFFu;
-        const int blk = ent & 0x1FFF;
-        const bool member = (ent & kPresent) && (((ent >> 13) & 3u) & rflag);
-        const int kvalid = member ? min(BK, N - blk * BK) : 0;
+        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+      } else if (kvalid > 0) {
 #pragma unroll
-        for (int c = 0; c < BK; ++c) {
-          const float x = c < kvalid ? s[e * BK + c] * scale_log2 : -INFINITY;
-          s[e * BK + c] = x;
-          mt = fmaxf(mt, x);
-        }
+        for (int c = 0; c < 64; ++c) mx = c < kvalid ? fmaxf(mx, s[c]) : mx;
       }
-      // running max with lazy rescale
+      red[(b * 2 + h) * 128 + r] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_red(b));
+      if (!__all_sync(full, wait(b_red(b), (t >> 1) & 1))) { ok = false; break; }
+      const float mo = red[(b * 2 + (h ^ 1)) * 128 + r];
+      const float mraw = fmaxf(mx, mo);
+      // running max (scaled, log2 domain) with lazy rescale
       bool rescale = false;
       float alpha = 1.f;
-      if (mt > -INFINITY) {
+      if (mraw > -INFINITY) {
+        const float mt = mraw * scale_log2;
         if (m_ref == -INFINITY) {
           m_ref = mt;
         } else if (mt > m_ref + kRescaleLog2) {
@@ -424,49 +483,53 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           rescale = true;
         }
       }
+      uint32_t pk[32];
       float rs = 0.f;
-      uint32_t pk[kTileN / 2];
+      if (kvalid > 0) {
 #pragma unroll
-      for (int c = 0; c < kTileN; c += 2) {
-        const float p0 = m_ref == -INFINITY ? 0.f : exp2f(s[c] - m_ref);
-        const float p1 = m_ref == -INFINITY ? 0.f : exp2f(s[c + 1] - m_ref);
-        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-        pk[c / 2] = *reinterpret_cast<uint32_t*>(&h);
-        // the row sum uses the rounded weights the MMA sees, so O / l is an
-        // exact convex combination of V rows
-        const float2 hr = __bfloat1622float2(h);
-        rs += hr.x + hr.y;
+        for (int c = 0; c < 64; c += 2) {
+          const float x0 = c < kvalid ? fmaf(s[c], scale_log2, -m_ref) : -INFINITY;
+          const float x1 = c + 1 < kvalid ? fmaf(s[c + 1], scale_log2, -m_ref) : -INFINITY;
+          __nv_bfloat162 hp = __floats2bfloat162_rn(fast_exp2(x0), fast_exp2(x1));
+          pk[c / 2] = *reinterpret_cast<uint32_t*>(&hp);
+          // the row sum uses the rounded weights the MMA sees, so O / l is
+          // an exact convex combination of V rows
+          const float2 hr = __bfloat1622float2(hp);
+          rs += hr.x + hr.y;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
       l += rs;
-      // P buffer b is free once PV of tile t-2 completed
-      if (t >= 2 && !__all_sync(0xffffffffu, wait(b_pv_done(b), ((t >> 1) & 1) ^ 1))) {
+      // P buffer b is free once P V of tile t-2 completed
+      if (t >= 2 && !__all_sync(full, wait(b_pv_done(b), ((t >> 1) & 1) ^ 1))) {
         ok = false;
         break;
       }
       uint8_t* prow = prow_base + b * kPBytes;
 #pragma unroll
-      for (int u = 0; u < kTileN / 8; ++u) {  // 16-byte units of 8 keys
-        const int ch = u / 8, uu = u % 8;
-        uint4 val = make_uint4(pk[u * 4], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
-        *reinterpret_cast<uint4*>(prow + ch * 16384 + ((uu ^ (r & 7)) << 4)) = val;
-      }
+      for (int u = 0; u < 8; ++u)  // 16-byte units of 8 keys, 128B swizzle
+        *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
+            make_uint4(pk[u * 4], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      // rescale O (warp-wide TMEM access) once the previous PV is complete
-      if (__any_sync(0xffffffffu, rescale)) {
-        if (t >= 1 && !__all_sync(0xffffffffu, wait(b_pv_done((t - 1) & 1), ((t - 1) >> 1) & 1))) {
+      // rescale this half of O (warp-wide TMEM access) once the previous
+      // P V is complete
+      if (__any_sync(full, rescale)) {
+        if (t >= 1 && !__all_sync(full, wait(b_pv_done((t - 1) & 1), ((t - 1) >> 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < DH; c += 32) {
           float o[32];
-          tmem_ld32(tO + lane_off + c, o);
+          tmem_ld32(tO + lane_off + h * DH + c, o);
           tmem_wait_ld();
           reg_fence<32>(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tO + lane_off + c, o);
+          tmem_st32(tO + lane_off + h * DH + c, o);
         }
         tmem_wait_st();
       }
@@ -474,18 +537,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(b_p_full(b));
     }
-    // epilogue: O / l, LSE
+    // epilogue: total row sum from both halves, O / l, LSE
+    const int fb = T & 1;  // red slot last used by tile T-2, read by all
+    red[(fb * 2 + h) * 128 + r] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_fin);
+    bool fin = ok && __all_sync(full, wait(b_fin, 0));
+    const float ltot = fin ? l + red[(fb * 2 + (h ^ 1)) * 128 + r] : 0.f;
     const int row = qt * kTileM + r;
-    const i64 orow = (i64(bh) * N + row) * D;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    bool fin = ok && T > 0;  // warp-uniform
-    if (fin) fin = __all_sync(0xffffffffu, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
-    if (fin) {
+    const i64 orow = (i64(bh) * N + row) * D + h * DH;
+    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+    if (fin && T > 0) fin = __all_sync(full, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
+    if (fin && T > 0) {
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < DH; c += 32) {
         float o[32];
-        tmem_ld32(tO + lane_off + c, o);
+        tmem_ld32(tO + lane_off + h * DH + c, o);
         tmem_wait_ld();
         reg_fence<32>(o);
         if (row < N) {
@@ -496,11 +564,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
     } else if (row < N) {
-      for (int c = 0; c < D; c += 4)
+      for (int c = 0; c < DH; c += 4)
         *reinterpret_cast<float4*>(o_s + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (row < N)
-      lse[i64(bh) * N + row] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (row < N && h == 0)
+      lse[i64(bh) * N + row] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
   }
 
   // teardown: on an abort let in-flight copies and MMAs drain (bounded)
@@ -549,7 +617,7 @@ bool make_map(CUtensorMap* m, const void* ptr, const Geom& g, int rows) {
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return static_cast<size_t>(D / 64) * 16384 * (1 + 2 * kStages) + 2 * 32768 + 256 + 1024;
+  return kSmemRequest;
 }
 
 template <int D, int BQ, int BK>
