@@ -30,6 +30,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace sla {
 
@@ -43,131 +44,6 @@ constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softma
 constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
-
-// ------------------------------------------------------------------ PTX
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            int z, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
-// columns [col, col+32) of TMEM lane (lane_base + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  uint32_t r[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// Values produced by tcgen05.ld may only be read after tcgen05.wait::ld; this
-// empty asm (ordered after the wait) re-defines them so no use of a loaded
-// value can be scheduled above the wait.
-template <int K>
-__device__ __forceinline__ void reg_fence(float* v) {
-#pragma unroll
-  for (int i = 0; i < K; ++i) asm volatile("" : "+f"(v[i]));
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// 2^x with the hardware approximation (ex2.approx, flush-to-zero): relative
-// error ~2^-22, far below the bf16 rounding P goes through next.
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
-// 1; addresses and byte offsets are encoded in 16-byte units.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
-         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator,
-// A/B K-major (0) or MN-major (1), N >> 3 at bit 17, M >> 4 at bit 24.
-constexpr uint32_t idesc_bf16(int m, int n, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
-         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
-         (static_cast<uint32_t>(m >> 4) << 24);
-}
 
 // ------------------------------------------------------------------ plan
 // One key-tile descriptor packs two 16-bit entries (the second only used for
@@ -227,13 +103,32 @@ __global__ void plan_kernel(sla_block_lists rows, int BH, int nqb, int nkb, int 
 
 // ------------------------------------------------------------------ kernel
 
+}  // namespace
+
+// What the kernel writes once the rows are done.  Sparse-only use writes
+// o_s; the fused forward writes `out` (bf16), adding the linear branch of
+// the tile's query blocks when `marg_cnt` is set: O_lin = phi(Q) H^M /
+// (phi(Q) . z^M) from the gathered summaries, then out = O_s + O_lin W.
+struct AttnEpilogue {
+  float* o_s;                 // [B*H, N, d] fp32, nullable
+  float* lse;                 // [B*H, N] fp32
+  __nv_bfloat16* out;         // [B*H, N, d] bf16, nullable
+  float* o_lin;               // [B*H, N, d] fp32, nullable (linear branch on)
+  const float* zm;            // [B*H*Nqb, 128] z^M (linear branch on)
+  const int32_t* marg_cnt;    // [B*H*Nqb] marginal counts; nullptr: branch off
+  int nqb;
+};
+
+namespace {
+
 template <int D, int BQ, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ plan_cnt,
-               const uint32_t* __restrict__ plan_tiles, int plan_stride, float* __restrict__ o_s,
-               float* __restrict__ lse, int32_t* status, int N, int nqt, float scale_log2,
-               long long timeout_cycles, int debug_skip) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmHM,
+               const __grid_constant__ CUtensorMap tmW, const int32_t* __restrict__ plan_cnt,
+               const uint32_t* __restrict__ plan_tiles, int plan_stride, AttnEpilogue ep,
+               int32_t* status, int N, int nqt, float scale_log2, long long timeout_cycles,
+               int debug_skip) {
   constexpr int DC = D / 64;                  // 64-element (128 B) chunks along d
   constexpr int DH = D / 2;                   // O columns per softmax half
   constexpr uint32_t kQBytes = DC * 16384;    // Q tile 128 x D bf16
@@ -266,8 +161,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto b_pv_done = [&](int b) { return smem_u32(&bars[15 + b]); };
   auto b_red = [&](int b) { return smem_u32(&bars[17 + b]); };
   const uint32_t b_fin = smem_u32(&bars[19]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[20]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[21]);
+  const uint32_t b_lin = smem_u32(&bars[20]);   // H^M and W tiles landed
+  const uint32_t b_phiq = smem_u32(&bars[21]);  // phi(Q) written (8 warps)
+  const uint32_t b_den = smem_u32(&bars[22]);   // normaliser halves exchanged (8 warps)
+  const uint32_t b_num = smem_u32(&bars[23]);   // phi(Q) H^M in TMEM
+  const uint32_t b_olin = smem_u32(&bars[24]);  // O_lin (bf16) in shared memory (8 warps)
+  const uint32_t b_lout = smem_u32(&bars[25]);  // O_lin W in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[26]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[27]);
   float* red = reinterpret_cast<float*>(base + offRed);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -275,6 +176,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int bh = tile / nqt, qt = tile % nqt;
   const int T = plan_cnt[tile];
   const uint32_t* ptiles = plan_tiles + i64(tile) * plan_stride;
+  // linear branch of this tile's query blocks (A: rows 0-63 or the whole
+  // 128-row block, B: rows 64-127 when blocks are 64 rows)
+  const int nqb = ep.nqb;
+  const int qa = BQ == 128 ? qt : 2 * qt;
+  const int qb2 = (BQ == 64 && 2 * qt + 1 < nqb) ? 2 * qt + 1 : -1;
+  int nm_a = 0, nm_b = 0;
+  if (D == 128 && ep.marg_cnt) {
+    nm_a = ep.marg_cnt[bh * nqb + qa];
+    if (qb2 >= 0) nm_b = ep.marg_cnt[bh * nqb + qb2];
+  }
+  const bool lin = nm_a > 0 || nm_b > 0;
 
   // The dynamic window must hold the 1024-aligned layout; it does whenever
   // the window starts 1024-aligned (then pad == 0).  Refuse otherwise.
@@ -299,6 +211,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(b_red(b), kSoftmaxWarps);
     }
     mbar_init(b_fin, kSoftmaxWarps);
+    mbar_init(b_lin, 1);
+    mbar_init(b_phiq, kSoftmaxWarps);
+    mbar_init(b_den, kSoftmaxWarps);
+    mbar_init(b_num, 1);
+    mbar_init(b_olin, kSoftmaxWarps);
+    mbar_init(b_lout, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -334,7 +252,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ---------------------------------------------------------- producer
     // K of tile t+2 may load once S of tile t has been computed; V of tile
     // t+2 once P V of tile t has: the two rings advance independently.
-    if (lane == 0 && T > 0) {
+    if (lane == 0 && (T > 0 || lin)) {
       mbar_expect_tx(b_q, kQBytes);
 #pragma unroll
       for (int c = 0; c < DC; ++c) tma_load_3d(sb + offQ + c * 16384, &tmQ, c * 64, qt * kTileM, bh, b_q);
@@ -375,6 +293,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (*abort_flag) break;
           if (clock64() - t0 > timeout_cycles) { give_up(); break; }
         }
+      }
+      // linear branch: H^M of the tile's query blocks and W go into the K/V
+      // stages once the last P V product has read them
+      if (lin && tv == T && (T == 0 || wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1))) {
+        mbar_expect_tx(b_lin, (nm_a > 0 ? 32768u : 0u) + (nm_b > 0 ? 32768u : 0u) + 32768u);
+        if (nm_a > 0) {
+          tma_load_2d(sb + offK, &tmHM, 0, (bh * nqb + qa) * 128, b_lin);
+          tma_load_2d(sb + offK + 16384, &tmHM, 64, (bh * nqb + qa) * 128, b_lin);
+        }
+        if (nm_b > 0) {
+          tma_load_2d(sb + offK + kKBytes, &tmHM, 0, (bh * nqb + qb2) * 128, b_lin);
+          tma_load_2d(sb + offK + kKBytes + 16384, &tmHM, 64, (bh * nqb + qb2) * 128, b_lin);
+        }
+        tma_load_2d(sb + offV, &tmW, 0, 0, b_lin);
+        tma_load_2d(sb + offV + 16384, &tmW, 64, 0, b_lin);
       }
     }
   } else if (warp == 1) {
@@ -418,6 +351,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int t = 0; ok && t < T; ++t) {
         if (t + 1 < T) ok = issue_s(t + 1);
         if (ok) ok = issue_pv(t);
+      }
+    }
+    if (lane == 0 && lin) {
+      bool ok = wait(b_lin, 0) && wait(b_phiq, 0);
+      if (ok) {
+        // num = phi(Q) H^M: M = 128 rows, N = 128 channels, K = 128 (A = phi(Q)
+        // K-major in the Q tile, B = H^M rows of channels, MN-major)
+        tc_fence_after();
+        constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+        for (int q2 = 0; q2 < 2; ++q2) {
+          if ((q2 == 0 ? nm_a : nm_b) <= 0) continue;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+            tc_mma(tS[q2], sdesc(sb + offQ + off, 16, 1024),
+                   sdesc(sb + offK + q2 * kKBytes + kk * 2048, 16384, 1024), idesc, kk > 0);
+          }
+        }
+        tc_commit(b_num);
+        ok = wait(b_olin, 0);
+      }
+      if (ok) {
+        // O_lin W: A = O_lin (bf16, K-major, in P buffer 0), B = W (MN-major)
+        tc_fence_after();
+        constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          tc_mma(tS[0], sdesc(sb + offP + off, 16, 1024), sdesc(sb + offV + kk * 2048, 16384, 1024),
+                 idesc, kk > 0);
+        }
+        tc_commit(b_lout);
       }
     }
   } else {
@@ -547,28 +512,120 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int row = qt * kTileM + r;
     const i64 orow = (i64(bh) * N + row) * D + h * DH;
     const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+    // all P V products done: O final in TMEM, Q, P and the S columns free
     if (fin && T > 0) fin = __all_sync(full, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
-    if (fin && T > 0) {
-      tc_fence_after();
+    bool lin_ok = false;
+    if (D == 128 && lin && fin) {  // (never taken for d = 64: lin is false)
+      // phi(Q) in place (this thread: row r, channels [64h, 64h + 64)), and
+      // half of the normaliser phi(q) . z^M from the same rounded values
+      const bool second = BQ == 64 && r >= 64;
+      const int nm_r = second ? nm_b : nm_a;
+      const float* zrow = ep.zm + (i64(bh) * nqb + (second ? qb2 : qa)) * 128 + h * 64;
+      float dpart = 0.f;
+      lin_ok = __all_sync(full, wait(b_q, 0));
+      if (lin_ok) {
 #pragma unroll
-      for (int c = 0; c < DH; c += 32) {
-        float o[32];
+        for (int u = 0; u < 8; ++u) {
+          uint4* p = reinterpret_cast<uint4*>(base + offQ + h * 16384 + sw128(r, u));
+          uint4 val = make_uint4(0u, 0u, 0u, 0u);
+          if (row < N && nm_r > 0) {
+            val = phi_unit(*p);
+            const uint32_t w4[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+              dpart = fmaf(f.x, __ldg(zrow + u * 8 + 2 * e), dpart);
+              dpart = fmaf(f.y, __ldg(zrow + u * 8 + 2 * e + 1), dpart);
+            }
+          }
+          *p = val;
+        }
+        const int db = fb ^ 1;  // slot of tile T-1, read by all before b_fin
+        red[(db * 2 + h) * 128 + r] = dpart;
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) { mbar_arrive(b_phiq); mbar_arrive(b_den); }
+        lin_ok = __all_sync(full, wait(b_den, 0));
+      }
+      float den = 0.f;
+      if (lin_ok) den = dpart + red[((fb ^ 1) * 2 + (h ^ 1)) * 128 + r];
+      if (lin_ok) lin_ok = __all_sync(full, wait(b_num, 0));
+      if (lin_ok) {
+        // O_lin = phi(Q) H^M / den -> o_lin (fp32, optional) and bf16 into P
+        // buffer 0 as the A operand of the projection
+        tc_fence_after();
+        const uint32_t tn = second ? tS[1] : tS[0];
+        const float dinv = (nm_r > 0 && den > 0.f) ? 1.f / den : 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          float v[32];
+          tmem_ld32(tn + lane_off + h * 64 + c, v);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = nm_r > 0 ? v[i] * dinv : 0.f;  // TMEM unwritten when no list
+          if (ep.o_lin && row < N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(ep.o_lin + orow + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          }
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(base + offP + h * 16384 + sw128(r, c / 8 + q4)) =
+                make_uint4(pack_bf16x2(v[8 * q4], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                           pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_olin);
+        lin_ok = __all_sync(full, wait(b_lout, 0));
+        if (lin_ok) tc_fence_after();
+      }
+    } else if (ep.o_lin && row < N) {
+      for (int c = 0; c < DH; c += 4)
+        *reinterpret_cast<float4*>(ep.o_lin + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // final: O / l (+ O_lin W) -> out (bf16) and / or o_s (fp32)
+#pragma unroll
+    for (int c = 0; c < DH; c += 32) {
+      float o[32];
+      if (fin && T > 0) {
         tmem_ld32(tO + lane_off + h * DH + c, o);
         tmem_wait_ld();
         reg_fence<32>(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= inv;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      }
+      if (row < N && ep.o_s) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(ep.o_s + orow + c + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+      }
+      if (ep.out) {
+        if (D == 128 && lin_ok) {
+          float lo[32];
+          tmem_ld32(tS[0] + lane_off + h * DH + c, lo);
+          tmem_wait_ld();
+          reg_fence<32>(lo);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] += lo[i];
+        }
         if (row < N) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(o_s + orow + c + i) =
-                make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(ep.out + orow + c + 8 * q4) =
+                make_uint4(pack_bf16x2(o[8 * q4], o[8 * q4 + 1]), pack_bf16x2(o[8 * q4 + 2], o[8 * q4 + 3]),
+                           pack_bf16x2(o[8 * q4 + 4], o[8 * q4 + 5]), pack_bf16x2(o[8 * q4 + 6], o[8 * q4 + 7]));
         }
       }
-    } else if (row < N) {
-      for (int c = 0; c < DH; c += 4)
-        *reinterpret_cast<float4*>(o_s + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (row < N && h == 0)
-      lse[i64(bh) * N + row] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
+      ep.lse[i64(bh) * N + row] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
   }
 
   // teardown: on an abort let in-flight copies and MMAs drain (bounded)
@@ -586,62 +643,53 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 // ------------------------------------------------------------------ host
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 // [B*H, N, d] bf16 viewed as a 3D tensor (d fastest); box of 64 x rows x 1
 // with 128-byte swizzle, rows past N read as zeros.
 bool make_map(CUtensorMap* m, const void* ptr, const Geom& g, int rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.N),
-                        static_cast<cuuint64_t>(g.BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.d) * 2,
-                           static_cast<cuuint64_t>(g.N) * g.d * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-template <int D>
-constexpr size_t smem_bytes() {
-  return kSmemRequest;
+  const uint64_t dims[3] = {static_cast<uint64_t>(g.d), static_cast<uint64_t>(g.N),
+                            static_cast<uint64_t>(g.BH)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(g.d) * 2, static_cast<uint64_t>(g.N) * g.d * 2};
+  const uint32_t box[3] = {64, static_cast<uint32_t>(rows), 1};
+  return encode_bf16_map(m, ptr, 3, dims, strides, box);
 }
 
 template <int D, int BQ, int BK>
 cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const int32_t* cnt, const uint32_t* tiles, const Geom& g, int nqt, float* o_s,
-                     float* lse, int32_t* status, cudaStream_t s) {
+                     const CUtensorMap& mhm, const CUtensorMap& mw, const int32_t* cnt,
+                     const uint32_t* tiles, const Geom& g, int nqt, const AttnEpilogue& ep,
+                     int32_t* status, cudaStream_t s) {
   auto kern = attn_tc_kernel<D, BQ, BK>;
-  const size_t smem = smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                                       static_cast<int>(kSmemRequest));
   if (e != cudaSuccess) return e;
   const float scale_log2 = g.scale * 1.4426950408889634f;
   const bool debug = (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0;
   const long long timeout = debug ? (1ll << 24) : (1ll << 31);
-  kern<<<g.BH * nqt, kThreads, smem, s>>>(mq, mk, mv, cnt, tiles, g.nkb, o_s, lse, status, g.N,
-                                          nqt, scale_log2, timeout, debug ? 1 : 0);
+  kern<<<g.BH * nqt, kThreads, kSmemRequest, s>>>(mq, mk, mv, mhm, mw, cnt, tiles, g.nkb, ep, status,
+                                                  g.N, nqt, scale_log2, timeout, debug ? 1 : 0);
   return cudaGetLastError();
+}
+
+struct PlanPtrs {
+  int32_t* cnt;
+  uint32_t* tiles;
+};
+
+PlanPtrs plan_ptrs(const Geom& g, void* scratch) {
+  const int nqt = (g.N + kTileM - 1) / kTileM;
+  const size_t ntiles = static_cast<size_t>(g.BH) * nqt;
+  PlanPtrs p;
+  p.cnt = static_cast<int32_t*>(scratch);
+  p.tiles = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) +
+                                        ((ntiles * sizeof(int32_t) + 255) & ~size_t(255)));
+  return p;
 }
 
 }  // namespace
 
 bool attn_tc_supported(const Geom& g) {
   return g.dtype == SLA_BF16 && (g.d == 64 || g.d == 128) && (g.bq == 64 || g.bq == 128) &&
-         (g.bk == 64 || g.bk == 128) && encode_fn() != nullptr;
+         (g.bk == 64 || g.bk == 128) && tma_available();
 }
 
 size_t attn_tc_scratch_bytes(const Geom& g) {
@@ -650,24 +698,47 @@ size_t attn_tc_scratch_bytes(const Geom& g) {
   return tiles * sizeof(int32_t) + 256 + tiles * g.nkb * sizeof(uint32_t);
 }
 
-cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const Geom& g,
-                           const sla_block_lists& rows, float* o_s, float* lse, int32_t* status,
-                           void* scratch, cudaStream_t s) {
+cudaError_t launch_attn_plan(const Geom& g, const sla_block_lists& rows, void* scratch,
+                             cudaStream_t s) {
   const int nqt = (g.N + kTileM - 1) / kTileM;
   const size_t ntiles = static_cast<size_t>(g.BH) * nqt;
-  int32_t* cnt = static_cast<int32_t*>(scratch);
-  uint32_t* tiles = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) +
-                                                ((ntiles * sizeof(int32_t) + 255) & ~size_t(255)));
+  const PlanPtrs pp = plan_ptrs(g, scratch);
   plan_kernel<<<static_cast<unsigned>((ntiles + 127) / 128), 128, 0, s>>>(
-      rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, cnt, tiles);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  CUtensorMap mq, mk, mv;
+      rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, pp.cnt, pp.tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tc_fused(const void* q, const void* k, const void* v, const Geom& g,
+                                 void* scratch, const AttnOutputs& o, const LinInputs* lin,
+                                 int32_t* status, cudaStream_t s) {
+  const int nqt = (g.N + kTileM - 1) / kTileM;
+  const PlanPtrs pp = plan_ptrs(g, scratch);
+  CUtensorMap mq, mk, mv, mhm, mw;
   if (!make_map(&mq, q, g, kTileM) || !make_map(&mk, k, g, g.bk) || !make_map(&mv, v, g, g.bk))
     return cudaErrorInvalidValue;
-#define SLA_TC_CASE(D_, BQ_, BK_)                                                              \
-  if (g.d == D_ && g.bq == BQ_ && g.bk == BK_)                                                 \
-    return launch_t<D_, BQ_, BK_>(mq, mk, mv, cnt, tiles, g, nqt, o_s, lse, status, s);
+  AttnEpilogue ep;
+  ep.o_s = o.o_s;
+  ep.lse = o.lse;
+  ep.out = static_cast<__nv_bfloat16*>(o.out);
+  ep.o_lin = o.o_lin;
+  ep.zm = nullptr;
+  ep.marg_cnt = nullptr;
+  ep.nqb = g.nqb;
+  mhm = mq;  // unused unless the linear branch is fused
+  mw = mq;
+  if (lin) {
+    if (g.d != 128) return cudaErrorNotSupported;
+    const uint64_t dh[2] = {128, static_cast<uint64_t>(g.BH) * g.nqb * 128}, sh[1] = {256};
+    const uint64_t dw[2] = {128, 128}, sw[1] = {256};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_bf16_map(&mhm, lin->hm, 2, dh, sh, box) || !encode_bf16_map(&mw, lin->wb, 2, dw, sw, box))
+      return cudaErrorInvalidValue;
+    ep.zm = lin->zm;
+    ep.marg_cnt = lin->marg_cnt;
+  }
+#define SLA_TC_CASE(D_, BQ_, BK_)                                                                 \
+  if (g.d == D_ && g.bq == BQ_ && g.bk == BK_)                                                    \
+    return launch_t<D_, BQ_, BK_>(mq, mk, mv, mhm, mw, pp.cnt, pp.tiles, g, nqt, ep, status, s);
   SLA_TC_CASE(128, 64, 64)
   SLA_TC_CASE(128, 64, 128)
   SLA_TC_CASE(128, 128, 64)
@@ -678,6 +749,19 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const Ge
   SLA_TC_CASE(64, 128, 128)
 #undef SLA_TC_CASE
   return cudaErrorNotSupported;
+}
+
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const Geom& g,
+                           const sla_block_lists& rows, float* o_s, float* lse, int32_t* status,
+                           void* scratch, cudaStream_t s) {
+  cudaError_t e = launch_attn_plan(g, rows, scratch, s);
+  if (e != cudaSuccess) return e;
+  AttnOutputs o;
+  o.o_s = o_s;
+  o.lse = lse;
+  o.out = nullptr;
+  o.o_lin = nullptr;
+  return launch_attn_tc_fused(q, k, v, g, scratch, o, nullptr, status, s);
 }
 
 }  // namespace sla

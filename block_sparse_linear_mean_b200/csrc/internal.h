@@ -30,6 +30,11 @@ constexpr double kFixedOne = 4611686018427387904.0;  // 2^62
 constexpr float kTieEps = 1e-5f;
 constexpr int kMaxBlocks = 8192;                     // Nqb, Nkb limit
 
+// TMA descriptors (tma_host.cu)
+bool tma_available();
+bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box);
+
 // mask path
 cudaError_t launch_pool(const void* x, int dtype, float* out, int BH, int N,
                         int d, int block, cudaStream_t s);
@@ -53,12 +58,46 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v,
                            float* o_s, float* lse, int32_t* status,
                            void* scratch, cudaStream_t s);
 size_t attn_tc_scratch_bytes(const Geom& g);
+// Outputs of the fused tensor-core attention; any pointer may be null.
+struct AttnOutputs {
+  float* o_s;     // fp32 O_s
+  float* lse;     // fp32 LSE (required)
+  void* out;      // bf16 out = O_s (+ O_lin W when the linear branch is fused)
+  float* o_lin;   // fp32 O_lin
+};
+// Prepared linear-branch tensors (from launch_lin_tc_prepare).
+struct LinInputs {
+  const void* hm;          // bf16 H^M [B*H*Nqb, 128, 128]
+  const void* wb;          // bf16 W [128, 128]
+  const float* zm;         // fp32 z^M [B*H*Nqb, 128]
+  const int32_t* marg_cnt; // marginal list counts [B*H*Nqb]
+};
+cudaError_t launch_attn_plan(const Geom& g, const sla_block_lists& rows, void* scratch,
+                             cudaStream_t s);
+cudaError_t launch_attn_tc_fused(const void* q, const void* k, const void* v, const Geom& g,
+                                 void* scratch, const AttnOutputs& o, const LinInputs* lin,
+                                 int32_t* status, cudaStream_t s);
 cudaError_t launch_lin_summary(const void* k, const void* v, const Geom& g,
                                float* hsum, float* zsum, cudaStream_t s);
 cudaError_t launch_lin_apply(const void* q, const float* hsum,
                              const float* zsum, const sla_block_lists& rows,
                              const float* o_s, const float* proj, void* out,
                              float* o_lin, const Geom& g, cudaStream_t s);
+
+cudaError_t launch_combine_copy(const float* o_s, void* out, float* o_lin, const Geom& g,
+                                cudaStream_t s);
+
+// tensor-core linear branch (bf16, d = 128): linear_tc.cu
+bool lin_tc_supported(const Geom& g);
+size_t lin_tc_scratch_bytes(const Geom& g);
+cudaError_t launch_lin_tc(const void* q, const void* k, const void* v, const float* proj,
+                          const sla_block_lists& rows, const float* o_s, void* out,
+                          float* o_lin, const Geom& g, void* scratch, int32_t* status,
+                          cudaStream_t s);
+cudaError_t launch_lin_tc_prepare(const void* k, const void* v, const float* proj,
+                                  const sla_block_lists& rows, const Geom& g, void* scratch,
+                                  int32_t* status, cudaStream_t s);
+LinInputs lin_tc_inputs(const Geom& g, void* scratch, const sla_block_lists& rows);
 
 // backward
 cudaError_t launch_bwd_prep(const void* dout, const float* o_s,

@@ -182,7 +182,35 @@ cudaError_t apply_t(const void* q, const float* hsum, const float* zsum,
   return cudaGetLastError();
 }
 
+// Linear branch off: out = O_s in the output dtype, o_lin = 0 (8 elements
+// per thread, 32-byte fp32 reads).
+template <typename T>
+__global__ void combine_copy_kernel(const float* __restrict__ o_s, T* __restrict__ out,
+                                    float* __restrict__ o_lin, i64 n8) {
+  const i64 i = i64(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(o_s)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(o_s)[2 * i + 1];
+  store4(out + 8 * i, a);
+  store4(out + 8 * i + 4, b);
+  if (o_lin) {
+    reinterpret_cast<float4*>(o_lin)[2 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(o_lin)[2 * i + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_combine_copy(const float* o_s, void* out, float* o_lin, const Geom& g,
+                                cudaStream_t s) {
+  const i64 n8 = i64(g.BH) * g.N * g.d / 8;
+  const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
+  if (g.dtype == SLA_BF16)
+    combine_copy_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(o_s, static_cast<__nv_bfloat16*>(out), o_lin, n8);
+  else
+    combine_copy_kernel<float><<<blocks, 256, 0, s>>>(o_s, static_cast<float*>(out), o_lin, n8);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_lin_summary(const void* k, const void* v, const Geom& g,
                                float* hsum, float* zsum, cudaStream_t s) {

@@ -195,18 +195,23 @@ __device__ void compact_row(const int8_t* lab, int n, int32_t* idx_c,
 }
 
 // ---------------------------------------------------------------------------
-// Classifier: one CTA per (bh, query block) row.
-//   1. P = softmax of the row's logits (fp32, fixed reduction order);
-//   2. sort 64-bit keys (P bits << 32 | ~index) descending -- rank order is
-//      score descending, block index ascending on equal scores;
-//   3. top-k: first n_c ranks critical, next n_m marginal;
-//      CDF: tail sums of P over the ranks in exact 2^-62 fixed point (integer
-//      adds, order-free), a rank is dropped iff its tail sum (itself and all
-//      lower ranks) is below thr; the top rank is always kept;
-//   4. write the mask row and the ascending CSR lists; count near-ties.
+// Classifier: one CTA (256 threads) per (bh, query block) row.
+//   1. P = softmax of the row's logits (fp32, fixed reduction order), kept as
+//      32-bit patterns: scores are non-negative, so the patterns order like
+//      the values;
+//   2. rank order is score descending, block index ascending on equal
+//      scores; no sort is needed, only the scores at the cuts:
+//      top-k: radix selection (4 passes of 8-bit digits, per-warp histograms)
+//      finds the score v at rank k and how many scores exceed it; among the
+//      blocks scoring exactly v the lowest indices fill the remaining slots;
+//      CDF: the same passes over exact 2^-62 fixed-point sums (integer adds,
+//      order-free) find the score at which the running tail sum -- a block
+//      plus every lower-ranked block -- first reaches thr; blocks below it
+//      are dropped, the top rank is always kept;
+//   3. write the mask row and the ascending CSR lists; count near-ties.
 
 struct ClassifyArgs {
-  int nkb, S, mode, n_c, n_m;
+  int nkb, mode, n_c, n_m;
   int from_prob;  // input rows are already softmaxed scores, not logits
   uint64_t thr_fx;
   int8_t* mask;
@@ -215,21 +220,195 @@ struct ClassifyArgs {
   int32_t* tie_count;
 };
 
-__device__ __forceinline__ uint64_t to_fixed(float p) {
-  return __double2ull_rz(static_cast<double>(p) * kFixedOne);
+__device__ __forceinline__ uint64_t to_fixed(uint32_t pbits) {
+  return __double2ull_rz(static_cast<double>(__uint_as_float(pbits)) * kFixedOne);
+}
+
+struct SelShared {
+  uint32_t hist[8][256];
+  unsigned long long hsum[8][256];
+  uint32_t tot[256];
+  unsigned long long tots[256];
+  uint32_t res_u[4];
+  unsigned long long res_l[4];
+};
+
+// Rank-k score (k counted from the top, 0-based) among the n patterns: the
+// value v and the number of patterns strictly above it.
+__device__ void select_rank(const uint32_t* pb, int n, int k, SelShared& sh, uint32_t& v,
+                            int& above) {
+  const int tid = threadIdx.x, w = tid / 32, lane = tid % 32;
+  uint32_t prefix = 0, mask = 0;
+  int krem = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 8 * 256; b += kCT) (&sh.hist[0][0])[b] = 0u;
+    __syncthreads();
+    for (int j = tid; j < n; j += kCT) {
+      const uint32_t x = pb[j];
+      if ((x & mask) == prefix) atomicAdd(&sh.hist[w][(x >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    {
+      uint32_t t = 0;
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) t += sh.hist[ww][tid];
+      sh.tot[tid] = t;
+    }
+    __syncthreads();
+    if (w == 0) {  // lanes walk bins from the top, 8 each
+      uint32_t c[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { c[i] = sh.tot[255 - 8 * lane - i]; local += c[i]; }
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - local;
+      const bool here = excl <= static_cast<uint32_t>(krem) && static_cast<uint32_t>(krem) < incl;
+      if (here) {
+        uint32_t acc = excl;
+        for (int i = 0; i < 8; ++i) {
+          if (static_cast<uint32_t>(krem) < acc + c[i]) {
+            sh.res_u[0] = 255 - 8 * lane - i;
+            sh.res_u[1] = acc;
+            break;
+          }
+          acc += c[i];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= sh.res_u[0] << shift;
+    mask |= 255u << shift;
+    krem -= static_cast<int>(sh.res_u[1]);
+    __syncthreads();
+  }
+  v = prefix;
+  above = k - krem;
+}
+
+// CDF cut: the score v* of the lowest-ranked kept block and the fixed-point
+// mass strictly below v* ("below"), or found = false when the whole row's
+// mass stays under thr.
+__device__ void select_mass(const uint32_t* pb, int n, uint64_t thr, SelShared& sh, uint32_t& v,
+                            uint64_t& below, bool& found) {
+  const int tid = threadIdx.x, w = tid / 32, lane = tid % 32;
+  uint32_t prefix = 0, mask = 0;
+  uint64_t blw = 0;
+  found = true;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 8 * 256; b += kCT) (&sh.hsum[0][0])[b] = 0ull;
+    __syncthreads();
+    for (int j = tid; j < n; j += kCT) {
+      const uint32_t x = pb[j];
+      if ((x & mask) == prefix)
+        atomicAdd(&sh.hsum[w][(x >> shift) & 255u], static_cast<unsigned long long>(to_fixed(x)));
+    }
+    __syncthreads();
+    {
+      unsigned long long t = 0;
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) t += sh.hsum[ww][tid];
+      sh.tots[tid] = t;
+    }
+    __syncthreads();
+    if (w == 0) {  // lanes walk bins from the bottom, 8 each
+      unsigned long long c[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { c[i] = sh.tots[8 * lane + i]; local += c[i]; }
+      unsigned long long incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned long long excl = incl - local;
+      // first bin whose cumulative mass (with everything below) reaches thr
+      const bool here = blw + excl < thr && thr <= blw + incl;
+      if (lane == 31 && blw + incl < thr) { sh.res_u[0] = 0xFFFFFFFFu; }
+      if (here) {
+        unsigned long long acc = excl;
+        for (int i = 0; i < 8; ++i) {
+          if (thr <= blw + acc + c[i]) {
+            sh.res_u[0] = 8 * lane + i;
+            sh.res_l[0] = acc;
+            break;
+          }
+          acc += c[i];
+        }
+      }
+      if (thr <= blw && lane == 0) {  // already reached (thr = 0): lowest bin
+        for (int i = 0; i < 256; ++i) if (sh.tots[i]) { sh.res_u[0] = i; sh.res_l[0] = 0; break; }
+      }
+    }
+    __syncthreads();
+    if (sh.res_u[0] == 0xFFFFFFFFu) { found = false; __syncthreads(); return; }
+    prefix |= sh.res_u[0] << shift;
+    mask |= 255u << shift;
+    blw += sh.res_l[0];
+    __syncthreads();
+  }
+  v = prefix;
+  below = blw;
+}
+
+// Largest pattern strictly below v (0 if none).
+__device__ uint32_t max_below(const uint32_t* pb, int n, uint32_t v, uint32_t* redu) {
+  uint32_t m = 0;
+  for (int j = threadIdx.x; j < n; j += kCT) {
+    const uint32_t x = pb[j];
+    if (x < v && x > m) m = x;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();
+  if (threadIdx.x % 32 == 0) redu[threadIdx.x / 32] = m;
+  __syncthreads();
+  uint32_t r = 0;
+  for (int i = 0; i < kCT / 32; ++i) r = max(r, redu[i]);
+  return r;
+}
+
+// Label pass: in index order, a block is in the top `take` ranks when its
+// pattern exceeds v, or equals v and fewer than `fill` lower-indexed blocks
+// also equal v.  `lab` gets `val` for those (and keeps larger labels).
+__device__ void label_top(const uint32_t* pb, int n, uint32_t v, int fill, int8_t* lab,
+                          int8_t val, int* wsum) {
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  int base = 0;
+  for (int j0 = 0; j0 < n; j0 += kCT) {
+    const int j = j0 + threadIdx.x;
+    const uint32_t x = j < n ? pb[j] : 0u;
+    const bool eq = j < n && x == v;
+    const unsigned be = __ballot_sync(0xffffffffu, eq);
+    __syncthreads();
+    if (l == 0) wsum[w] = __popc(be);
+    __syncthreads();
+    int off = base, tot = 0;
+    for (int i = 0; i < kCT / 32; ++i) {
+      if (i < w) off += wsum[i];
+      tot += wsum[i];
+    }
+    const int rank_eq = off + __popc(be & ((1u << l) - 1u));
+    if (j < n && (x > v || (eq && rank_eq < fill)) && lab[j] < val) lab[j] = val;
+    base += tot;
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__ logits,
                                                        ClassifyArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
-  int8_t* lab = reinterpret_cast<int8_t*>(keys + a.S);
+  const int nkb = a.nkb, tid = threadIdx.x;
+  uint32_t* pb = reinterpret_cast<uint32_t*>(smem);
+  int8_t* lab = reinterpret_cast<int8_t*>(pb + nkb);
+  __shared__ SelShared sh;
   __shared__ float redf[32];
   __shared__ int redi[32];
-  __shared__ uint64_t seg_suffix[kCT];
-  __shared__ uint64_t t_at[2];
+  __shared__ uint32_t redu[32];
   const int row = blockIdx.x;
-  const int nkb = a.nkb, S = a.S, tid = threadIdx.x;
   const float* lr = logits + i64(row) * nkb;
 
   // 1. softmax over the row (skipped for rows given as scores)
@@ -243,115 +422,119 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
     se = block_reduce_sum(se, redf);
     inv = 1.0f / se;
   }
-  for (int j = tid; j < S; j += kCT) {
-    uint64_t key = 0;
-    if (j < nkb) {
-      // scores are non-negative, so their bit patterns order like the values
-      const float p = a.from_prob ? fmaxf(lr[j], 0.f) : expf(lr[j] - m) * inv;
-      if (a.scores) a.scores[i64(row) * nkb + j] = p;
-      key = (static_cast<uint64_t>(__float_as_uint(p)) << 32) |
-            static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(j));
-    }
-    keys[j] = key;
+  for (int j = tid; j < nkb; j += kCT) {
+    const float p = a.from_prob ? fmaxf(lr[j], 0.f) : expf(lr[j] - m) * inv;
+    if (a.scores) a.scores[i64(row) * nkb + j] = p;
+    pb[j] = __float_as_uint(p);
+    lab[j] = 0;
   }
   __syncthreads();
 
-  // 2. bitonic sort, descending
-  for (int k = 2; k <= S; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = tid; i < S; i += kCT) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const uint64_t x = keys[i], y = keys[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (x < y) : (x > y)) { keys[i] = y; keys[ixj] = x; }
+  // 2. cuts
+  bool tie = false;
+  int c = 0;  // critical (kept) count
+  if (a.mode == SLA_MASK_TOPK) {
+    c = a.n_c;
+    if (c > 0) {
+      uint32_t v;
+      int above;
+      select_rank(pb, nkb, c - 1, sh, v, above);
+      label_top(pb, nkb, v, c - above, lab, 2, redi);
+      if (a.tie_count && c < nkb) {  // gap between ranks c-1 and c
+        const uint32_t nxt = max_below(pb, nkb, v, redu);
+        // rank c shares v when v's group is not exhausted by the cut
+        int eqcount = 0;
+        for (int j = tid; j < nkb; j += kCT) eqcount += pb[j] == v;
+        eqcount = block_reduce_sum_int(eqcount, redi);
+        const float hi = __uint_as_float(v);
+        const float lo = (above + eqcount > c) ? hi : __uint_as_float(nxt);
+        tie |= (hi - lo) <= kTieEps * hi;
+      }
+    }
+  } else {
+    uint32_t v = 0;
+    uint64_t below = 0;
+    bool found = false;
+    if (a.thr_fx > 0) select_mass(pb, nkb, a.thr_fx, sh, v, below, found);
+    if (a.thr_fx == 0) {
+      for (int j = tid; j < nkb; j += kCT) lab[j] = 2;  // nothing can be dropped
+      c = nkb;
+      __syncthreads();
+    } else {
+      uint32_t vk;
+      int fill;
+      if (found) {
+        // group of blocks scoring exactly v: with r = ceil((thr - below) / fx(v))
+        // the r lowest-ranked (highest-index) ones are still below thr when
+        // taken alone, the other g - r + 1 are kept
+        int g = 0;
+        for (int j = tid; j < nkb; j += kCT) g += pb[j] == v;
+        g = block_reduce_sum_int(g, redi);
+        const uint64_t fx = to_fixed(v);
+        const uint64_t r = (a.thr_fx - below + fx - 1) / fx;
+        vk = v;
+        fill = g - static_cast<int>(r) + 1;
+      } else {
+        // the row's whole mass stays below thr: only the top rank is kept
+        uint32_t mx = 0;
+        for (int j = tid; j < nkb; j += kCT) mx = max(mx, pb[j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        __syncthreads();
+        if (tid % 32 == 0) redu[tid / 32] = mx;
+        __syncthreads();
+        mx = 0;
+        for (int i = 0; i < kCT / 32; ++i) mx = max(mx, redu[i]);
+        vk = mx;
+        fill = 1;
+      }
+      label_top(pb, nkb, vk, fill, lab, 2, redi);
+      int above = 0, eqc = 0;
+      for (int j = tid; j < nkb; j += kCT) { above += pb[j] > vk; eqc += pb[j] == vk; }
+      above = block_reduce_sum_int(above, redi);
+      eqc = block_reduce_sum_int(eqc, redi);
+      c = above + fill;
+      if (a.tie_count && found) {
+        const double thr = static_cast<double>(a.thr_fx) / kFixedOne;
+        const uint64_t fx = to_fixed(vk);
+        const uint64_t r = static_cast<uint64_t>(eqc - fill + 1);   // kept block's tail count
+        const double t_last = static_cast<double>(below + r * fx) / kFixedOne;
+        const double t_next = static_cast<double>(below + (r - 1) * fx) / kFixedOne;
+        if (c > 1) tie |= fabs(t_last - thr) <= kTieEps;
+        if (c < nkb) {
+          tie |= fabs(thr - t_next) <= kTieEps;
+          const float hi = __uint_as_float(vk);
+          const float lo = r >= 2 ? hi : __uint_as_float(max_below(pb, nkb, vk, redu));
+          tie |= (hi - lo) <= kTieEps * hi;
         }
       }
-      __syncthreads();
     }
   }
-
-  // 3. number of critical ranks
-  int c = a.n_c;
-  const int seg = S / kCT;  // ranks per thread (S >= kCT)
-  if (a.mode == SLA_MASK_CDF) {
-    uint64_t local = 0;
-    for (int r = tid * seg; r < (tid + 1) * seg; ++r)
-      if (r < nkb) local += to_fixed(__uint_as_float(static_cast<uint32_t>(keys[r] >> 32)));
-    seg_suffix[tid] = local;
-    __syncthreads();
-    if (tid < 32) {  // suffix sums of the 256 segment totals, one warp
-      uint64_t v8[8], tot = 0;
-      for (int e = 0; e < 8; ++e) { v8[e] = seg_suffix[tid * 8 + e]; tot += v8[e]; }
-      uint64_t incl = tot;  // inclusive suffix over lanes >= tid
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint64_t y = __shfl_down_sync(0xffffffffu, incl, o);
-        if (tid + o < 32) incl += y;
-      }
-      uint64_t run = incl - tot;  // lanes > tid
-      for (int e = 7; e >= 0; --e) { seg_suffix[tid * 8 + e] = run; run += v8[e]; }
-    }
-    __syncthreads();
-    int kept = 0;
-    uint64_t run = seg_suffix[tid];
-    for (int r = (tid + 1) * seg - 1; r >= tid * seg; --r) {
-      if (r >= nkb) continue;
-      run += to_fixed(__uint_as_float(static_cast<uint32_t>(keys[r] >> 32)));
-      if (run >= a.thr_fx) ++kept;
-    }
-    c = block_reduce_sum_int(kept, redi);
-    if (c < 1) c = 1;
-    // record the two decisive tail sums for the tie report
-    if (a.tie_count) {
-      run = seg_suffix[tid];
-      for (int r = (tid + 1) * seg - 1; r >= tid * seg; --r) {
-        if (r >= nkb) continue;
-        run += to_fixed(__uint_as_float(static_cast<uint32_t>(keys[r] >> 32)));
-        if (r == c - 1) t_at[0] = run;
-        if (r == c) t_at[1] = run;
-      }
-    }
-  }
+  // marginal: the next n_m ranks after the c critical ones
   const int nm = min(a.n_m, nkb - c);
-  // labels by rank
-  for (int r = tid; r < nkb; r += kCT) {
-    const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(keys[r]));
-    lab[j] = r < c ? 2 : (r < c + nm ? 1 : 0);
+  if (nm > 0) {
+    uint32_t v;
+    int above;
+    select_rank(pb, nkb, c + nm - 1, sh, v, above);
+    label_top(pb, nkb, v, c + nm - above, lab, 1, redi);
+    if (a.tie_count && c + nm < nkb) {
+      const uint32_t nxt = max_below(pb, nkb, v, redu);
+      int eqcount = 0;
+      for (int j = tid; j < nkb; j += kCT) eqcount += pb[j] == v;
+      eqcount = block_reduce_sum_int(eqcount, redi);
+      const float hi = __uint_as_float(v);
+      const float lo = (above + eqcount > c + nm) ? hi : __uint_as_float(nxt);
+      tie |= (hi - lo) <= kTieEps * hi;
+    }
   }
+  if (a.tie_count && tid == 0 && tie) atomicAdd(a.tie_count, 1);
   __syncthreads();
 
-  // tie report: the decisive margins of this row, as seen in fp32 P -- score
-  // gaps at a cut relative to the higher score, tail sums against thr in
-  // absolute (unit mass) terms
-  if (a.tie_count && tid == 0) {
-    auto pr = [&](int r) { return __uint_as_float(static_cast<uint32_t>(keys[r] >> 32)); };
-    auto close = [&](int r) { return (pr(r) - pr(r + 1)) <= kTieEps * pr(r); };
-    bool tie = false;
-    if (a.mode == SLA_MASK_TOPK) {
-      if (c > 0 && c < nkb) tie |= close(c - 1);
-    } else if (a.thr_fx > 0) {
-      const double thr = static_cast<double>(a.thr_fx) / kFixedOne;
-      if (c > 1) tie |= fabs(static_cast<double>(t_at[0]) / kFixedOne - thr) <= kTieEps;
-      if (c < nkb) {
-        tie |= fabs(thr - static_cast<double>(t_at[1]) / kFixedOne) <= kTieEps;
-        tie |= close(c - 1);
-      }
-    }
-    if (nm > 0 && c + nm < nkb) tie |= close(c + nm - 1);
-    if (tie) atomicAdd(a.tie_count, 1);
-  }
-
-  // 4. mask row and lists
+  // 3. mask row and lists
   for (int j = tid; j < nkb; j += kCT) a.mask[i64(row) * nkb + j] = lab[j];
   const i64 off = i64(row) * nkb;
   compact_row(lab, nkb, a.rows.crit_idx + off, a.rows.crit_cnt + row,
               a.rows.marg_idx + off, a.rows.marg_cnt + row, redi);
-}
-
-static int sort_size(int n) {
-  int s = kCT;
-  while (s < n) s <<= 1;
-  return s;
 }
 
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
@@ -360,7 +543,6 @@ cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
   ClassifyArgs a;
   a.from_prob = from_prob ? 1 : 0;
   a.nkb = g.nkb;
-  a.S = sort_size(g.nkb);
   a.mode = g.mode;
   a.n_c = g.n_c;
   a.n_m = g.n_m;
@@ -369,7 +551,7 @@ cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
   a.rows = rows;
   a.scores = scores;
   a.tie_count = tie_count;
-  const size_t smem = static_cast<size_t>(a.S) * 8 + static_cast<size_t>(a.S);
+  const size_t smem = static_cast<size_t>(g.nkb) * 5 + 16;
   cudaError_t e = cudaFuncSetAttribute(classify_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

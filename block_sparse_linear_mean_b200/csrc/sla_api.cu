@@ -71,7 +71,7 @@ bool has_linear_branch(const Geom& g) { return g.linear; }
 
 // Workspace layouts (each region 256-byte aligned).
 struct MaskWs { size_t qbar, kbar, logits, total; };
-struct FwdWs { size_t o_s, hsum, zsum, tc, total; };
+struct FwdWs { size_t o_s, hsum, zsum, lintc, tc, total; };
 struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, total; };
 
 MaskWs mask_ws(const Geom& g) {
@@ -88,10 +88,14 @@ FwdWs fwd_ws(const Geom& g) {
   FwdWs w;
   size_t off = kStatusBytes;
   w.o_s = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.N * g.d);
-  w.hsum = w.zsum = off;
+  w.hsum = w.zsum = w.lintc = off;
   if (has_linear_branch(g)) {
-    w.hsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d * g.d);
-    w.zsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+    if (sla::lin_tc_supported(g)) {
+      w.lintc = off; off = align_up(off + sla::lin_tc_scratch_bytes(g));
+    } else {
+      w.hsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d * g.d);
+      w.zsum = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+    }
   }
   w.tc = off; off = align_up(off + sla::attn_tc_scratch_bytes(g));
   w.total = off;
@@ -265,22 +269,54 @@ sla_status sla_linear_combine(const sla_params* p, const void* q, const void* k,
   const FwdWs w = fwd_ws(g);
   if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* hsum = nullptr;
-  float* zsum = nullptr;
-  if (has_linear_branch(g)) {
-    hsum = at<float>(ws, w.hsum);
-    zsum = at<float>(ws, w.zsum);
-    SLA_CUDA(sla::launch_lin_summary(k, v, g, hsum, zsum, s));
+  if (!has_linear_branch(g)) {
+    SLA_CUDA(sla::launch_combine_copy(o_s, out, o_lin, g, s));
+    return SLA_OK;
   }
+  if (sla::lin_tc_supported(g)) {
+    SLA_CUDA(sla::launch_lin_tc(q, k, v, proj, *rows, o_s, out, o_lin, g, at<void>(ws, w.lintc),
+                                at<int32_t>(ws, 0), s));
+    return SLA_OK;
+  }
+  float* hsum = at<float>(ws, w.hsum);
+  float* zsum = at<float>(ws, w.zsum);
+  SLA_CUDA(sla::launch_lin_summary(k, v, g, hsum, zsum, s));
   SLA_CUDA(sla::launch_lin_apply(q, hsum, zsum, *rows, o_s, proj, out, o_lin, g, s));
   return SLA_OK;
 }
 
-sla_status sla_forward(const sla_params* p, const void* q, const void* k,
-                       const void* v, const float* proj,
-                       const sla_block_lists* rows, void* out, float* lse,
-                       float* o_s, float* o_lin, void* ws, size_t ws_bytes,
-                       void* stream) {
+static bool tc_attention(const Geom& g) {
+  return g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g);
+}
+
+sla_status sla_forward_prepare(const sla_params* p, const void* k, const void* v,
+                               const float* proj, const sla_block_lists* rows, void* ws,
+                               size_t ws_bytes, void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!tensor_ok(k) || !tensor_ok(v) || !tensor_ok(proj) || !tensor_ok(ws) || !lists_ok(rows))
+    return SLA_ERR_INVALID_ARG;
+  const FwdWs w = fwd_ws(g);
+  if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
+  if (tc_attention(g)) SLA_CUDA(sla::launch_attn_plan(g, *rows, at<void>(ws, w.tc), s));
+  if (has_linear_branch(g)) {
+    if (sla::lin_tc_supported(g))
+      SLA_CUDA(sla::launch_lin_tc_prepare(k, v, proj, *rows, g, at<void>(ws, w.lintc),
+                                          at<int32_t>(ws, 0), s));
+    else
+      SLA_CUDA(sla::launch_lin_summary(k, v, g, at<float>(ws, w.hsum), at<float>(ws, w.zsum), s));
+  }
+  return SLA_OK;
+}
+
+sla_status sla_attention_combine(const sla_params* p, const void* q, const void* k,
+                                 const void* v, const float* proj,
+                                 const sla_block_lists* rows, void* out, float* lse,
+                                 float* o_s, float* o_lin, void* ws, size_t ws_bytes,
+                                 void* stream) {
   Geom g;
   sla_status st = make_geom(p, &g);
   if (st != SLA_OK) return st;
@@ -290,10 +326,49 @@ sla_status sla_forward(const sla_params* p, const void* q, const void* k,
     return SLA_ERR_INVALID_ARG;
   const FwdWs w = fwd_ws(g);
   if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool linear = has_linear_branch(g);
+  int32_t* status = at<int32_t>(ws, 0);
+  if (tc_attention(g) && (!linear || sla::lin_tc_supported(g))) {
+    // one fused kernel: attention, linear apply, projection, combine
+    sla::AttnOutputs o;
+    o.o_s = o_s;
+    o.lse = lse;
+    o.out = out;
+    o.o_lin = o_lin;
+    sla::LinInputs li = sla::lin_tc_inputs(g, at<void>(ws, w.lintc), *rows);
+    SLA_CUDA(sla::launch_attn_tc_fused(q, k, v, g, at<void>(ws, w.tc), o, linear ? &li : nullptr,
+                                       status, s));
+    return SLA_OK;
+  }
   float* os = o_s ? o_s : at<float>(ws, w.o_s);
-  st = sla_sparse_attention(p, q, k, v, rows, os, lse, ws, ws_bytes, stream);
+  if (tc_attention(g)) {
+    sla::AttnOutputs o;
+    o.o_s = os;
+    o.lse = lse;
+    o.out = nullptr;
+    o.o_lin = nullptr;
+    SLA_CUDA(sla::launch_attn_tc_fused(q, k, v, g, at<void>(ws, w.tc), o, nullptr, status, s));
+  } else {
+    SLA_CUDA(sla::launch_attn_simt(q, k, v, g, *rows, os, lse, s));
+  }
+  if (!linear) {
+    SLA_CUDA(sla::launch_combine_copy(os, out, o_lin, g, s));
+  } else {
+    SLA_CUDA(sla::launch_lin_apply(q, at<float>(ws, w.hsum), at<float>(ws, w.zsum), *rows, os, proj,
+                                   out, o_lin, g, s));
+  }
+  return SLA_OK;
+}
+
+sla_status sla_forward(const sla_params* p, const void* q, const void* k,
+                       const void* v, const float* proj,
+                       const sla_block_lists* rows, void* out, float* lse,
+                       float* o_s, float* o_lin, void* ws, size_t ws_bytes,
+                       void* stream) {
+  sla_status st = sla_forward_prepare(p, k, v, proj, rows, ws, ws_bytes, stream);
   if (st != SLA_OK) return st;
-  return sla_linear_combine(p, q, k, v, proj, rows, os, out, o_lin, ws, ws_bytes, stream);
+  return sla_attention_combine(p, q, k, v, proj, rows, out, lse, o_s, o_lin, ws, ws_bytes, stream);
 }
 
 sla_status sla_backward(const sla_params* p, const void* q, const void* k,

@@ -38,7 +38,8 @@ SLA_FLAG_DEBUG_TIMEOUT = 2
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",
            "sla_workspace_size", "sla_build_mask", "sla_classify_scores",
            "sla_mask_lists",
-           "sla_forward", "sla_sparse_attention", "sla_sparse_attention_noalloc",
+           "sla_forward", "sla_forward_prepare", "sla_attention_combine",
+           "sla_sparse_attention", "sla_sparse_attention_noalloc",
            "sla_linear_combine",
            "sla_backward", "sla_forward_uses_tensor_cores",
            "sla_check_device_status")
@@ -95,6 +96,11 @@ def lib():
         L.sla_forward.restype = ctypes.c_int
         L.sla_forward.argtypes = [P(sla_params), VP, VP, VP, VP, P(sla_block_lists),
                                   VP, VP, VP, VP, VP, SZ, VP]
+        L.sla_forward_prepare.restype = ctypes.c_int
+        L.sla_forward_prepare.argtypes = [P(sla_params), VP, VP, VP, P(sla_block_lists), VP, SZ, VP]
+        L.sla_attention_combine.restype = ctypes.c_int
+        L.sla_attention_combine.argtypes = [P(sla_params), VP, VP, VP, VP, P(sla_block_lists),
+                                            VP, VP, VP, VP, VP, SZ, VP]
         L.sla_sparse_attention.restype = ctypes.c_int
         L.sla_sparse_attention.argtypes = [P(sla_params), VP, VP, VP, P(sla_block_lists),
                                            VP, VP, VP, SZ, VP]
@@ -163,6 +169,17 @@ def sla_mask_lists(p, mask, rows, cols, stream) -> int:
 def sla_forward(p, q, k, v, proj, rows, out, lse, o_s, o_lin, ws, ws_bytes, stream) -> int:
     return lib().sla_forward(ctypes.byref(p), q, k, v, proj, ctypes.byref(rows), out,
                              lse, o_s, o_lin, ws, ws_bytes, stream)
+
+
+def sla_forward_prepare(p, k, v, proj, rows, ws, ws_bytes, stream) -> int:
+    return lib().sla_forward_prepare(ctypes.byref(p), k, v, proj, ctypes.byref(rows), ws,
+                                     ws_bytes, stream)
+
+
+def sla_attention_combine(p, q, k, v, proj, rows, out, lse, o_s, o_lin, ws, ws_bytes,
+                          stream) -> int:
+    return lib().sla_attention_combine(ctypes.byref(p), q, k, v, proj, ctypes.byref(rows), out,
+                                       lse, o_s, o_lin, ws, ws_bytes, stream)
 
 
 def sla_sparse_attention(p, q, k, v, rows, o_s, lse, ws, ws_bytes, stream) -> int:

@@ -178,6 +178,23 @@ SLA_API sla_status sla_forward(const sla_params* p, const void* q, const void* k
                        float* o_s, float* o_lin, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* sla_forward in two stages (sla_forward = prepare, then combine, on the same
+ * workspace and lists).  Prepare: the per-query-tile key-block plan of the
+ * tensor-core attention and, with the linear branch on, the key-block
+ * summaries H_j, z_j and their per-query-block sums H^M, z^M.  It resets the
+ * workspace status word.  Combine: the attention over critical blocks, the
+ * linear attention over marginal blocks, the projection and the sum -- for
+ * bf16 with d = 128 (or the linear branch off) one fused kernel that writes
+ * `out` directly.  Arguments as for sla_forward. */
+SLA_API sla_status sla_forward_prepare(const sla_params* p, const void* k, const void* v,
+                               const float* proj, const sla_block_lists* rows, void* ws,
+                               size_t ws_bytes, void* stream);
+SLA_API sla_status sla_attention_combine(const sla_params* p, const void* q, const void* k,
+                                 const void* v, const float* proj,
+                                 const sla_block_lists* rows, void* out, float* lse,
+                                 float* o_s, float* o_lin, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /* Step 4, critical part alone (NABLA-style sparse attention):
  *   o_s        [B,H,N,d] fp32 out: softmax attention over each query block's
  *              critical key blocks (0 where the block has none)

@@ -1,0 +1,66 @@
+"""The GPU classifier on crafted score rows (sla_classify_scores), bit for bit
+against the oracle on the very same fp32 values: exact duplicates (index
+tie-break), zeros, tiny and wide rows, and CDF rows whose dyadic masses put
+tail sums exactly on thr (the strict 'exceeds 1 - thr' boundary)."""
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_linear_mean_b200 import sla, synth
+from gpu_util import expected_rows, lists_from_gpu
+from oracle import sla_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+
+def _rows(kind, nkb, nrows, rng):
+    if kind == "dups":
+        p = rng.choice([1.0, 2.0, 3.0, 5.0, 8.0], size=(nrows, nkb))
+    elif kind == "zeros":
+        p = rng.random((nrows, nkb)) ** 6
+        p[rng.random((nrows, nkb)) < 0.5] = 0.0
+        p[:, 0] += 1e-3
+    elif kind == "dyadic":
+        p = 2.0 ** -rng.integers(1, 12, size=(nrows, nkb)).astype(np.float64)
+    else:
+        p = rng.random((nrows, nkb)) ** 4
+    p = p / p.sum(axis=1, keepdims=True)
+    return p.astype(np.float32)
+
+
+def _params(nkb, nrows, mode, fc=0.0, fm=0.0, thr=0.0):
+    wl = synth.Workload(name="cls", B=1, H=1, grid=(1, 1, nkb * 64), d=64, dtype="f32",
+                        block_q=64, block_k=64, mode=mode, frac_crit=fc, frac_marg=fm, thr=thr)
+    p = sla.params_for(wl)
+    # one head of nrows query blocks: N spans max(nrows, nkb) blocks of 64
+    return wl, p
+
+
+@pytest.mark.parametrize("kind", ["dups", "zeros", "dyadic", "smooth"])
+@pytest.mark.parametrize("nkb", [1, 7, 64, 300, 1920])
+@pytest.mark.parametrize("mode,fc,fm,thr", [("topk", 0.05, 0.10, 0.0), ("topk", 0.5, 0.25, 0.0),
+                                            ("cdf", 0.0, 0.0, 0.2), ("cdf", 0.0, 0.1, 0.5),
+                                            ("cdf", 0.0, 0.0, 0.0)])
+def test_classifier_bit_exact_on_crafted_rows(kind, nkb, mode, fc, fm, thr):
+    rng = np.random.default_rng(nkb * 7 + len(kind))
+    nrows = nkb  # square: Nqb = Nkb
+    s32 = _rows(kind, nkb, nrows, rng)
+    wl, p = _params(nkb, nrows, mode, fc, fm, thr)
+    got = sla.classify_scores(p, torch.from_numpy(s32.reshape(1, 1, nrows, nkb)).cuda())
+    torch.cuda.synchronize()
+    mask = got["mask"].cpu().numpy()[0, 0]
+    ref, margins = orc.classify(s32.astype(np.float64), mode, fc, fm, thr)
+    if mode == "topk":
+        np.testing.assert_array_equal(mask, ref)
+    else:
+        # the decision may differ only where a tail sum lies within 1e-12 of
+        # thr (fixed point vs binary64 summation order); dyadic rows are exact
+        diff = (mask != ref).any(axis=-1)
+        assert not (diff & (margins > 1e-12)).any()
+        if kind == "dyadic":
+            np.testing.assert_array_equal(mask, ref)
+    assert lists_from_gpu(got["rows"], nrows, nkb) == expected_rows(mask[None, None])
+    # the GPU's own tie count equals the oracle's on the same values
+    if mode == "topk" or kind == "dyadic":
+        assert int(got["ties"].item()) == int((margins <= 1e-5).sum())
