@@ -38,7 +38,7 @@ namespace {
 
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 8;                 // two warpgroups
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softmax
 constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
@@ -133,14 +133,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   constexpr int DH = D / 2;                   // O columns per softmax half
   constexpr uint32_t kQBytes = DC * 16384;    // Q tile 128 x D bf16
   constexpr uint32_t kKBytes = DC * 16384;    // K (or V) tile 128 x D
-  constexpr uint32_t kPBytes = 2 * 16384;     // P tile 128 x 128 bf16
   constexpr uint32_t offQ = 0;
   constexpr uint32_t offK = offQ + kQBytes;
   constexpr uint32_t offV = offK + kStages * kKBytes;
-  constexpr uint32_t offP = offV + kStages * kKBytes;
-  constexpr uint32_t offRed = offP + 2 * kPBytes;      // [2 parity][2 halves][128] fp32
+  constexpr uint32_t offOL = offK + 2 * kKBytes;       // O_lin (bf16) after the loop: K stage 2
+  constexpr uint32_t offRed = offV + kStages * kKBytes;  // [2 parity][2 halves][128] fp32
   constexpr uint32_t offBar = offRed + 2 * 2 * 128 * 4;
-  constexpr uint32_t kUsed = offBar + 256;
+  constexpr uint32_t kUsed = offBar + 512;
   constexpr uint32_t idesc_qk = idesc_bf16(128, kTileN, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
 
@@ -150,25 +149,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* base = smem_raw + pad;
   const uint32_t sb = raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
+  constexpr int kB0 = 1 + 4 * kStages;            // first barrier after the K/V rings
+  static_assert((kB0 + 20) * 8 <= kUsed - offBar, "barrier block too small");
   const uint32_t b_q = smem_u32(&bars[0]);
   auto b_k_full = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto b_v_full = [&](int s) { return smem_u32(&bars[3 + s]); };
-  auto b_k_empty = [&](int s) { return smem_u32(&bars[5 + s]); };
-  auto b_v_empty = [&](int s) { return smem_u32(&bars[7 + s]); };
-  auto b_s_full = [&](int b) { return smem_u32(&bars[9 + b]); };
-  auto b_s_free = [&](int b) { return smem_u32(&bars[11 + b]); };
-  auto b_p_full = [&](int b) { return smem_u32(&bars[13 + b]); };
-  auto b_pv_done = [&](int b) { return smem_u32(&bars[15 + b]); };
-  auto b_red = [&](int b) { return smem_u32(&bars[17 + b]); };
-  const uint32_t b_fin = smem_u32(&bars[19]);
-  const uint32_t b_lin = smem_u32(&bars[20]);   // H^M and W tiles landed
-  const uint32_t b_phiq = smem_u32(&bars[21]);  // phi(Q) written (8 warps)
-  const uint32_t b_den = smem_u32(&bars[22]);   // normaliser halves exchanged (8 warps)
-  const uint32_t b_num = smem_u32(&bars[23]);   // phi(Q) H^M in TMEM
-  const uint32_t b_olin = smem_u32(&bars[24]);  // O_lin (bf16) in shared memory (8 warps)
-  const uint32_t b_lout = smem_u32(&bars[25]);  // O_lin W in TMEM
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[26]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[27]);
+  auto b_v_full = [&](int s) { return smem_u32(&bars[1 + kStages + s]); };
+  auto b_k_empty = [&](int s) { return smem_u32(&bars[1 + 2 * kStages + s]); };
+  auto b_v_empty = [&](int s) { return smem_u32(&bars[1 + 3 * kStages + s]); };
+  auto b_s_full = [&](int b) { return smem_u32(&bars[kB0 + b]); };
+  auto b_s_free = [&](int b) { return smem_u32(&bars[kB0 + 2 + b]); };
+  auto b_p_full = [&](int b) { return smem_u32(&bars[kB0 + 4 + b]); };
+  auto b_pv_done = [&](int b) { return smem_u32(&bars[kB0 + 6 + b]); };
+  auto b_red = [&](int b) { return smem_u32(&bars[kB0 + 8 + b]); };
+  const uint32_t b_fin = smem_u32(&bars[kB0 + 10]);
+  const uint32_t b_lin = smem_u32(&bars[kB0 + 11]);   // H^M and W tiles landed
+  const uint32_t b_phiq = smem_u32(&bars[kB0 + 12]);  // phi(Q) written (8 warps)
+  const uint32_t b_den = smem_u32(&bars[kB0 + 13]);   // normaliser halves exchanged (8 warps)
+  const uint32_t b_num = smem_u32(&bars[kB0 + 14]);   // phi(Q) H^M in TMEM
+  const uint32_t b_olin = smem_u32(&bars[kB0 + 15]);  // O_lin (bf16) in shared memory (8 warps)
+  const uint32_t b_lout = smem_u32(&bars[kB0 + 16]);  // O_lin W in TMEM
+  // every P V product done (single use).  The producer cannot wait on
+  // pv_done for this: with more than two stages the completion before the
+  // last one on the same barrier may still be pending, and a parity wait
+  // would then take the older phase for the newer one.
+  const uint32_t b_pv_last = smem_u32(&bars[kB0 + 17]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB0 + 18]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB0 + 19]);
   float* red = reinterpret_cast<float*>(base + offRed);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -217,6 +223,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(b_num, 1);
     mbar_init(b_olin, kSoftmaxWarps);
     mbar_init(b_lout, 1);
+    mbar_init(b_pv_last, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -231,6 +238,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO = tmem + 256;
+  const uint32_t tP[2] = {tmem + 384, tmem + 448};  // bf16 P, two keys per column
 
   auto give_up = [&]() {
     *abort_flag = 1;
@@ -296,7 +304,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       // linear branch: H^M of the tile's query blocks and W go into the K/V
       // stages once the last P V product has read them
-      if (lin && tv == T && (T == 0 || wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1))) {
+      if (lin && tv == T && (T == 0 || wait(b_pv_last, 0))) {
         mbar_expect_tx(b_lin, (nm_a > 0 ? 32768u : 0u) + (nm_b > 0 ? 32768u : 0u) + 32768u);
         if (nm_a > 0) {
           tma_load_2d(sb + offK, &tmHM, 0, (bh * nqb + qa) * 128, b_lin);
@@ -335,14 +343,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!wait(b_p_full(b), (t >> 1) & 1)) return false;
         if (!wait(b_v_full(s), (t / kStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t pbase = sb + offP + b * kPBytes;
         const uint32_t vbase = sb + offV + s * kKBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk) {
-          const uint32_t poff = (kk / 4) * 16384 + (kk % 4) * 32;
-          tc_mma(tO, sdesc(pbase + poff, 16, 1024), sdesc(vbase + kk * 2048, 16384, 1024),
-                 idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
+          tc_mma_ts(tO, tP[b] + kk * 8, sdesc(vbase + kk * 2048, 16384, 1024), idesc_pv,
+                    (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(b_v_empty(s));
         tc_commit(b_pv_done(b));
         return true;
@@ -352,6 +357,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (t + 1 < T) ok = issue_s(t + 1);
         if (ok) ok = issue_pv(t);
       }
+      if (ok) tc_commit(b_pv_last);
     }
     if (lane == 0 && lin) {
       bool ok = wait(b_lin, 0) && wait(b_phiq, 0);
@@ -373,13 +379,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = wait(b_olin, 0);
       }
       if (ok) {
-        // O_lin W: A = O_lin (bf16, K-major, in P buffer 0), B = W (MN-major)
+        // O_lin W: A = O_lin (bf16, K-major, in K stage 2), B = W (MN-major)
         tc_fence_after();
         constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          tc_mma(tS[0], sdesc(sb + offP + off, 16, 1024), sdesc(sb + offV + kk * 2048, 16384, 1024),
+          tc_mma(tS[0], sdesc(sb + offOL + off, 16, 1024), sdesc(sb + offV + kk * 2048, 16384, 1024),
                  idesc, kk > 0);
         }
         tc_commit(b_lout);
@@ -399,7 +405,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const unsigned full = 0xffffffffu;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow_base = base + offP + h * 16384 + r * 128;
     for (int t = 0; ok && t < T; ++t) {
       const int b = t & 1;
       const uint32_t desc = ptiles[t];
@@ -472,12 +477,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = false;
         break;
       }
-      uint8_t* prow = prow_base + b * kPBytes;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)  // 16-byte units of 8 keys, 128B swizzle
-        *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
-            make_uint4(pk[u * 4], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // P (bf16 pairs) into TMEM: this half's 64 keys are columns [32h, 32h + 32)
+      tc_fence_after();
+      tmem_st32u(tP[b] + lane_off + h * 32, pk);
       // rescale this half of O (warp-wide TMEM access) once the previous
       // P V is complete
       if (__any_sync(full, rescale)) {
@@ -496,8 +498,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
           tmem_st32(tO + lane_off + h * DH + c, o);
         }
-        tmem_wait_st();
       }
+      tmem_wait_st();  // P (and any rescaled O) stored
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_p_full(b));
@@ -512,7 +514,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int row = qt * kTileM + r;
     const i64 orow = (i64(bh) * N + row) * D + h * DH;
     const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-    // all P V products done: O final in TMEM, Q, P and the S columns free
+    // all P V products done: O final in TMEM, Q, the K/V stages and the S
+    // columns free
     if (fin && T > 0) fin = __all_sync(full, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
     bool lin_ok = false;
     if (D == 128 && lin && fin) {  // (never taken for d = 64: lin is false)
@@ -552,8 +555,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (lin_ok) den = dpart + red[((fb ^ 1) * 2 + (h ^ 1)) * 128 + r];
       if (lin_ok) lin_ok = __all_sync(full, wait(b_num, 0));
       if (lin_ok) {
-        // O_lin = phi(Q) H^M / den -> o_lin (fp32, optional) and bf16 into P
-        // buffer 0 as the A operand of the projection
+        // O_lin = phi(Q) H^M / den -> o_lin (fp32, optional) and bf16 into K
+        // stage 2 as the A operand of the projection
         tc_fence_after();
         const uint32_t tn = second ? tS[1] : tS[0];
         const float dinv = (nm_r > 0 && den > 0.f) ? 1.f / den : 0.f;
@@ -572,7 +575,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(base + offP + h * 16384 + sw128(r, c / 8 + q4)) =
+            *reinterpret_cast<uint4*>(base + offOL + h * 16384 + sw128(r, c / 8 + q4)) =
                 make_uint4(pack_bf16x2(v[8 * q4], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
                            pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
         }

@@ -107,6 +107,8 @@ def test_forward_matches_oracle_with_oracle_mask(case, simt):
     _, rows, _ = feed_mask(p, ref["mask"])
     f = sla.forward(p, t["q"], t["k"], t["v"], t["proj"], rows, save_for_backward=True)
     torch.cuda.synchronize()
+    st = sla.check_device_status(f["ws"])
+    assert st == sla.SLA_OK, sla.status_string(st)
     o = orc.forward(x.q, x.k, x.v, x.proj, ref["mask"], wl.block_q, wl.block_k)
     res = {}
     for key in ("o_s", "o_lin", "out"):
