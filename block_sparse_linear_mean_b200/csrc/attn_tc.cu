@@ -39,6 +39,9 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 3;
+// One pair in kPolyEvery of a full tile's exponentials is computed by a cubic
+// on the FMA pipe instead of the special-function unit (0: none).
+constexpr int kPolyEvery = 3;
 constexpr int kSoftmaxWarps = 8;                 // two warpgroups
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softmax
 constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
@@ -150,7 +153,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t sb = raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
   constexpr int kB0 = 1 + 4 * kStages;            // first barrier after the K/V rings
-  static_assert((kB0 + 20) * 8 <= kUsed - offBar, "barrier block too small");
+  static_assert((kB0 + 28) * 8 <= kUsed - offBar, "barrier block too small");
   const uint32_t b_q = smem_u32(&bars[0]);
   auto b_k_full = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto b_v_full = [&](int s) { return smem_u32(&bars[1 + kStages + s]); };
@@ -160,7 +163,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto b_s_free = [&](int b) { return smem_u32(&bars[kB0 + 2 + b]); };
   auto b_p_full = [&](int b) { return smem_u32(&bars[kB0 + 4 + b]); };
   auto b_pv_done = [&](int b) { return smem_u32(&bars[kB0 + 6 + b]); };
-  auto b_red = [&](int b) { return smem_u32(&bars[kB0 + 8 + b]); };
+  // partial row maxima exchanged between the two warps holding the same 32
+  // rows (one per column half): one barrier per (tile parity, lane quadrant)
+  auto b_red = [&](int b, int quad) { return smem_u32(&bars[kB0 + 18 + 4 * b + quad]); };
   const uint32_t b_fin = smem_u32(&bars[kB0 + 10]);
   const uint32_t b_lin = smem_u32(&bars[kB0 + 11]);   // H^M and W tiles landed
   const uint32_t b_phiq = smem_u32(&bars[kB0 + 12]);  // phi(Q) written (8 warps)
@@ -173,8 +178,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // last one on the same barrier may still be pending, and a parity wait
   // would then take the older phase for the newer one.
   const uint32_t b_pv_last = smem_u32(&bars[kB0 + 17]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB0 + 18]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB0 + 19]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB0 + 26]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB0 + 27]);
   float* red = reinterpret_cast<float*>(base + offRed);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -214,7 +219,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(b_s_free(b), kSoftmaxWarps);
       mbar_init(b_p_full(b), kSoftmaxWarps);
       mbar_init(b_pv_done(b), 1);
-      mbar_init(b_red(b), kSoftmaxWarps);
+      for (int q = 0; q < 4; ++q) mbar_init(b_red(b, q), 2);
     }
     mbar_init(b_fin, kSoftmaxWarps);
     mbar_init(b_lin, 1);
@@ -236,9 +241,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128};
+  // columns: S of tiles with parity b at 128 b, O at 256, bf16 P of parity b
+  // (two keys per column) at 384 + 64 b.  Computed, not indexed from an
+  // array, so no address goes through local memory.
+  auto tS = [&](int b) { return tmem + 128u * static_cast<uint32_t>(b); };
   const uint32_t tO = tmem + 256;
-  const uint32_t tP[2] = {tmem + 384, tmem + 448};  // bf16 P, two keys per column
+  auto tP = [&](int b) { return tmem + 384u + 64u * static_cast<uint32_t>(b); };
 
   auto give_up = [&]() {
     *abort_flag = 1;
@@ -331,7 +339,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          tc_mma(tS[b], sdesc(sb + offQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), idesc_qk,
+          tc_mma(tS(b), sdesc(sb + offQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), idesc_qk,
                  kk > 0);
         }
         tc_commit(b_s_full(b));
@@ -346,7 +354,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t vbase = sb + offV + s * kKBytes;
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
-          tc_mma_ts(tO, tP[b] + kk * 8, sdesc(vbase + kk * 2048, 16384, 1024), idesc_pv,
+          tc_mma_ts(tO, tP(b) + kk * 8, sdesc(vbase + kk * 2048, 16384, 1024), idesc_pv,
                     (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(b_v_empty(s));
         tc_commit(b_pv_done(b));
@@ -371,7 +379,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-            tc_mma(tS[q2], sdesc(sb + offQ + off, 16, 1024),
+            tc_mma(tS(q2), sdesc(sb + offQ + off, 16, 1024),
                    sdesc(sb + offK + q2 * kKBytes + kk * 2048, 16384, 1024), idesc, kk > 0);
           }
         }
@@ -385,7 +393,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          tc_mma(tS[0], sdesc(sb + offOL + off, 16, 1024), sdesc(sb + offV + kk * 2048, 16384, 1024),
+          tc_mma(tS(0), sdesc(sb + offOL + off, 16, 1024), sdesc(sb + offV + kk * 2048, 16384, 1024),
                  idesc, kk > 0);
         }
         tc_commit(b_lout);
@@ -417,26 +425,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!__all_sync(full, wait(b_s_full(b), (t >> 1) & 1))) { ok = false; break; }
       tc_fence_after();
       float s[64];
-      tmem_ld32(tS[b] + lane_off + h * 64, s);
-      tmem_ld32(tS[b] + lane_off + h * 64 + 32, s + 32);
+      tmem_ld32(tS(b) + lane_off + h * 64, s);
+      tmem_ld32(tS(b) + lane_off + h * 64 + 32, s + 32);
       tmem_wait_ld();
       reg_fence<64>(s);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_s_free(b));
-      // partial max of the raw scores over this thread's valid keys
+      // partial max of the raw scores over this thread's valid keys (four
+      // independent three-input chains)
       float mx = -INFINITY;
       if (kvalid == 64) {
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 64; c += 8) {
+          a0 = max3(a0, s[c], s[c + 1]);
+          a1 = max3(a1, s[c + 2], s[c + 3]);
+          a2 = max3(a2, s[c + 4], s[c + 5]);
+          a3 = max3(a3, s[c + 6], s[c + 7]);
+        }
+        mx = max3(a0, a1, fmaxf(a2, a3));
       } else if (kvalid > 0) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) mx = c < kvalid ? fmaxf(mx, s[c]) : mx;
       }
       red[(b * 2 + h) * 128 + r] = mx;
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_red(b));
-      if (!__all_sync(full, wait(b_red(b), (t >> 1) & 1))) { ok = false; break; }
+      if (lane == 0) mbar_arrive(b_red(b, quad));
+      if (!__all_sync(full, wait(b_red(b, quad), (t >> 1) & 1))) { ok = false; break; }
       const float mo = red[(b * 2 + (h ^ 1)) * 128 + r];
       const float mraw = fmaxf(mx, mo);
       // running max (scaled, log2 domain) with lazy rescale
@@ -453,25 +469,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           rescale = true;
         }
       }
+      // P = 2^(s * scale_log2 - m_ref) rounded to bf16.  The row sum uses the
+      // rounded weights the MMA sees, so O / l is an exact convex
+      // combination of V rows.
       uint32_t pk[32];
-      float rs = 0.f;
-      if (kvalid > 0) {
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
+      if (kvalid == 64) {
+        // every kPolyEvery-th pair of exponentials goes to the FMA pipe
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float x0 = c < kvalid ? fmaf(s[c], scale_log2, -m_ref) : -INFINITY;
-          const float x1 = c + 1 < kvalid ? fmaf(s[c + 1], scale_log2, -m_ref) : -INFINITY;
-          __nv_bfloat162 hp = __floats2bfloat162_rn(fast_exp2(x0), fast_exp2(x1));
-          pk[c / 2] = *reinterpret_cast<uint32_t*>(&hp);
-          // the row sum uses the rounded weights the MMA sees, so O / l is
-          // an exact convex combination of V rows
-          const float2 hr = __bfloat1622float2(hp);
-          rs += hr.x + hr.y;
+        for (int i = 0; i < 32; ++i) {
+          const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
+          const float2 e = (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1)
+                               ? exp2_poly2(x)
+                               : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          pk[i] = pack_bf16x2(e.x, e.y);
+        }
+      } else if (kvalid > 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
+          pk[i] = pack_bf16x2(2 * i < kvalid ? fast_exp2(x.x) : 0.f,
+                              2 * i + 1 < kvalid ? fast_exp2(x.y) : 0.f);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
       }
-      l += rs;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        acc0 = add2(acc0, make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
+        acc1 = add2(acc1, make_float2(__uint_as_float(pk[i + 1] << 16), __uint_as_float(pk[i + 1] & 0xFFFF0000u)));
+        acc2 = add2(acc2, make_float2(__uint_as_float(pk[i + 2] << 16), __uint_as_float(pk[i + 2] & 0xFFFF0000u)));
+        acc3 = add2(acc3, make_float2(__uint_as_float(pk[i + 3] << 16), __uint_as_float(pk[i + 3] & 0xFFFF0000u)));
+      }
+      acc0 = add2(add2(acc0, acc1), add2(acc2, acc3));
+      l += acc0.x + acc0.y;
       // P buffer b is free once P V of tile t-2 completed
       if (t >= 2 && !__all_sync(full, wait(b_pv_done(b), ((t >> 1) & 1) ^ 1))) {
         ok = false;
@@ -479,7 +513,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       // P (bf16 pairs) into TMEM: this half's 64 keys are columns [32h, 32h + 32)
       tc_fence_after();
-      tmem_st32u(tP[b] + lane_off + h * 32, pk);
+      tmem_st32u(tP(b) + lane_off + h * 32, pk);
       // rescale this half of O (warp-wide TMEM access) once the previous
       // P V is complete
       if (__any_sync(full, rescale)) {
@@ -558,7 +592,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // O_lin = phi(Q) H^M / den -> o_lin (fp32, optional) and bf16 into K
         // stage 2 as the A operand of the projection
         tc_fence_after();
-        const uint32_t tn = second ? tS[1] : tS[0];
+        const uint32_t tn = tS(second ? 1 : 0);
         const float dinv = (nm_r > 0 && den > 0.f) ? 1.f / den : 0.f;
 #pragma unroll
         for (int c = 0; c < 64; c += 32) {
@@ -612,7 +646,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (ep.out) {
         if (D == 128 && lin_ok) {
           float lo[32];
-          tmem_ld32(tS[0] + lane_off + h * DH + c, lo);
+          tmem_ld32(tS(0) + lane_off + h * DH + c, lo);
           tmem_wait_ld();
           reg_fence<32>(lo);
 #pragma unroll

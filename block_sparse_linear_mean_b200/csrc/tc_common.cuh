@@ -138,6 +138,58 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Paired fp32 arithmetic: one instruction does the work of two lanes.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
+      "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+      "add.rn.f32x2 %0, ra, rb;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe, relieving the special-function unit.
+// Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer j in
+// the low mantissa bits of the sum, f = x - j lies in [-1/2, 1/2], 2^f is a
+// cubic (near-minimax in relative error, 7.5e-5, fitted by exp2_poly_fit.py
+// beside this file), and j is added to the exponent field.  x is clamped
+// below at -126 so the exponent stays in range (2^-126 stands in for
+// anything smaller); x must be at most 127.  The error is far below the
+// bf16 rounding the result goes through next.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = add2(x, make_float2(kShift, kShift));
+  const float2 j = add2(t, make_float2(-kShift, -kShift));
+  const float2 f = add2(x, make_float2(-j.x, -j.y));
+  float2 p = fma2(f, make_float2(0.0551716648042202f, 0.0551716648042202f),
+                  make_float2(0.2426111251115799f, 0.2426111251115799f));
+  p = fma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = fma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
 // 1; addresses and byte offsets are encoded in 16-byte units.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
