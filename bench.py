@@ -108,6 +108,29 @@ def effective_flops(wl, mask_np, N=None):
     return fl + lin, pairs, fl, lin, apply
 
 
+def backward_flops(wl, mask_np):
+    """Algorithmic flops of one backward over ``mask_np``: 10*d per kept
+    critical token pair (S and dP recomputed, dV, dK, dQ), plus the linear
+    branch: per token of a query block with marginal blocks g = dO W^T,
+    dW += O_lin^T dO, d phi(q) and the dH^M, dz^M outer products
+    (8*d^2 + 4*d); per marginal (query block, key block) pair the scatter
+    of dH^M, dz^M (d^2 + d); per token of a key block that is marginal for
+    some query block dk, dv (4*d^2 + 2*d).  Returns (total, critical, linear)."""
+    d = wl.d
+    sq, sk = block_sizes(wl.N, wl.block_q), block_sizes(wl.N, wl.block_k)
+    crit = (mask_np == 2).astype(np.float64)
+    cfl = 10.0 * d * float(np.einsum("bhij,i,j->", crit, sq, sk))
+    lfl = 0.0
+    if wl.frac_marg > 0:
+        marg = (mask_np == 1)
+        nm = marg.sum(axis=-1).astype(np.float64)
+        tok = float(np.einsum("bhi,i->", (nm > 0).astype(np.float64), sq))
+        ktok = float(np.einsum("bhj,j->", (marg.sum(axis=-2) > 0).astype(np.float64), sk))
+        lfl = tok * (8.0 * d * d + 4.0 * d) + float(nm.sum()) * (d * d + d) + \
+            ktok * (4.0 * d * d + 2.0 * d)
+    return cfl + lfl, cfl, lfl
+
+
 # --------------------------------------------------------------- clocks
 
 
@@ -188,18 +211,28 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = synth.WORKLOADS[args.workload]
-    x = synth.make_inputs(wl, seed=rank, device=dev)
+    bwd = wl.backward
+    x = synth.make_inputs(wl, seed=rank, device=dev, with_dout=bwd)
     p = sla.params_for(wl)
     ws_m = sla.workspace(p, sla.SLA_OP_MASK, dev)
     ws_f = sla.workspace(p, sla.SLA_OP_FORWARD, dev)
+    ws_b = sla.workspace(p, sla.SLA_OP_BACKWARD, dev) if bwd else None
     N, nqb, nkb = wl.N, math.ceil(wl.N / wl.block_q), math.ceil(wl.N / wl.block_k)
     B, H, d = wl.B, wl.H, wl.d
     mask = torch.empty(B, H, nqb, nkb, dtype=torch.int8, device=dev)
     rows = sla.BlockLists.empty(B * H * nqb, nkb, dev)
     rc = rows.c()
+    # the fine-tune step also needs the column lists and the saved O_s, O_lin
+    cols = sla.BlockLists.empty(B * H * nkb, nqb, dev) if bwd else None
+    cc = cols.c() if bwd else None
     out = torch.empty_like(x.q)
-    o_s = torch.empty(x.q.shape, dtype=torch.float32, device=dev)
-    lse = torch.empty(x.q.shape[:-1], dtype=torch.float32, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    o_s = torch.empty(x.q.shape, **f32) if bwd else None
+    o_lin = torch.empty(x.q.shape, **f32) if bwd else None
+    lse = torch.empty(x.q.shape[:-1], **f32)
+    if bwd:
+        dq, dk, dv = (torch.empty(x.q.shape, **f32) for _ in range(3))
+        dproj = torch.empty(x.proj.shape, **f32)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
@@ -210,7 +243,7 @@ def run_ours(args, rank, world, local_rank):
 
     def stage_mask(q, k):
         chk("sla_build_mask", sla.sla_build_mask(p, q.data_ptr(), k.data_ptr(), mask.data_ptr(),
-                                                 rc, None, None, None, ws_m.data_ptr(),
+                                                 rc, cc, None, None, ws_m.data_ptr(),
                                                  ws_m.numel(), sp))
 
     def stage_prepare(k, v):
@@ -221,13 +254,24 @@ def run_ours(args, rank, world, local_rank):
     def stage_combine(q, k, v, dst):
         chk("sla_attention_combine", sla.sla_attention_combine(
             p, q.data_ptr(), k.data_ptr(), v.data_ptr(), x.proj.data_ptr(), rc,
-            dst.data_ptr(), lse.data_ptr(), None, None, ws_f.data_ptr(), ws_f.numel(), sp))
+            dst.data_ptr(), lse.data_ptr(), o_s.data_ptr() if bwd else None,
+            o_lin.data_ptr() if bwd else None, ws_f.data_ptr(), ws_f.numel(), sp))
+
+    def stage_backward(q, k, v, dout):
+        chk("sla_backward", sla.sla_backward(
+            p, q.data_ptr(), k.data_ptr(), v.data_ptr(), x.proj.data_ptr(), dout.data_ptr(),
+            rc, cc, o_s.data_ptr(), lse.data_ptr(), o_lin.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), dproj.data_ptr(), ws_b.data_ptr(), ws_b.numel(), sp))
 
     fused = sla.sla_forward_uses_tensor_cores(p) == 1 and (wl.frac_marg == 0 or wl.d == 128)
     # kernels per step: pool x2, logits, classify | plan (+ W to bf16, summaries,
     # indicator, gather GEMM) | fused attention (or attention + combine)
     launches_per_step = 4 + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
         + (1 if (not fused and wl.frac_marg > 0) else 0) + (1 if fused else 2)
+    if bwd:
+        # column lists | Delta and g, dW partials, dQ, dK dV, (summaries,
+        # linear dq, linear dk dv), dW reduction
+        launches_per_step += 1 + 5 + (3 if wl.frac_marg > 0 else 0)
 
 
     # warm-up (also fixes the mask used to count the algorithmic work)
@@ -235,11 +279,18 @@ def run_ours(args, rank, world, local_rank):
         stage_mask(x.q, x.k)
         stage_prepare(x.k, x.v)
         stage_combine(x.q, x.k, x.v, out)
+        if bwd:
+            stage_backward(x.q, x.k, x.v, x.dout)
     torch.cuda.synchronize(dev)
     assert sla.check_device_status(ws_f) == sla.SLA_OK
-    flops, pairs, crit_fl, lin_fl, apply_fl = effective_flops(wl, mask.cpu().numpy())
+    if bwd:
+        assert sla.check_device_status(ws_b) == sla.SLA_OK
+    mask_np = mask.cpu().numpy()
+    flops, pairs, crit_fl, lin_fl, apply_fl = effective_flops(wl, mask_np)
+    bwd_fl = backward_flops(wl, mask_np) if bwd else (0.0, 0.0, 0.0)
+    flops += bwd_fl[0]
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -254,13 +305,17 @@ def run_ours(args, rank, world, local_rank):
             e[2].record(stream)
             stage_combine(x.q, x.k, x.v, out)
             e[3].record(stream)
+            if bwd:
+                stage_backward(x.q, x.k, x.v, x.dout)
+            e[4].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     t_mask = [e[0].elapsed_time(e[1]) for e in ev]
     t_prep = [e[1].elapsed_time(e[2]) for e in ev]
     t_comb = [e[2].elapsed_time(e[3]) for e in ev]
-    total_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
+    t_bwd = [e[3].elapsed_time(e[4]) for e in ev]
+    total_ms = sum(e[0].elapsed_time(e[4]) for e in ev)
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -272,21 +327,28 @@ def run_ours(args, rank, world, local_rank):
     # pinned memory, mask + forward, D2H of the output, every step
     e2e = None
     if not args.no_e2e:
-        qh, kh, vh = (t.cpu().pin_memory() for t in (x.q, x.k, x.v))
+        ins = (x.q, x.k, x.v, x.dout) if bwd else (x.q, x.k, x.v)
+        hosts = [t.cpu().pin_memory() for t in ins]
+        devs = [torch.empty_like(t) for t in ins]
+        grads_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                   for t in ((dq, dk, dv, dproj) if bwd else ())]
         oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        qd, kd, vd = (torch.empty_like(x.q) for _ in range(3))
         ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
         for s in range(args.steps):
             flush.zero_()
             ee[s][0].record(stream)
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            qd, kd, vd = devs[:3]
             stage_mask(qd, kd)
             stage_prepare(kd, vd)
             stage_combine(qd, kd, vd, out)
             oh.copy_(out, non_blocking=True)
+            if bwd:
+                stage_backward(qd, kd, vd, devs[3])
+                for h_, d_ in zip(grads_h, (dq, dk, dv, dproj)):
+                    h_.copy_(d_, non_blocking=True)
             ee[s][1].record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
@@ -295,8 +357,9 @@ def run_ours(args, rank, world, local_rank):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = float(t.item())
         e2e = {"value": world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": int(3 * x.q.numel() * x.q.element_size()),
-               "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in ins)),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size() +
+                                         sum(t.numel() * t.element_size() for t in grads_h)),
                "ms_per_step": e2e_ms / args.steps}
 
     peaks, peak_src = load_peaks()
@@ -333,9 +396,12 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "256 MB write flushes L2 between steps, outside the timed events"},
         "breakdown_ms": {"mask": round(statistics.mean(t_mask), 4),
                          "prepare (plan + linear summaries + gather)": round(statistics.mean(t_prep), 4),
-                         "attention_combine": round(comb_ms, 4)},
+                         "attention_combine": round(comb_ms, 4),
+                         **({"backward": round(statistics.mean(t_bwd), 4)} if bwd else {})},
         "work": {"effective_flops_per_step": flops, "critical_flops": crit_fl,
                  "linear_flops": lin_fl, "critical_token_pairs": pairs,
+                 **({"backward_critical_flops": bwd_fl[1], "backward_linear_flops": bwd_fl[2]}
+                    if bwd else {}),
                  "kept_fraction_of_dense_pairs": pairs / (B * H * float(N) * N)},
         "roofline": roofline,
         "e2e": e2e,

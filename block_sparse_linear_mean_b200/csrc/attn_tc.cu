@@ -54,7 +54,7 @@ constexpr float kRescaleLog2 = 8.0f;
 // block of rows 0-63, bit 14: rows 64-127; both for a 128-row block), bits
 // 0-12 key-block index.
 
-constexpr uint32_t kPresent = 1u << 15;
+constexpr uint32_t kPresent = kPlanPresent;
 
 __device__ __forceinline__ uint32_t entry(int blk, uint32_t flags) {
   return kPresent | (flags << 13) | static_cast<uint32_t>(blk);
@@ -742,6 +742,16 @@ cudaError_t launch_attn_plan(const Geom& g, const sla_block_lists& rows, void* s
   const PlanPtrs pp = plan_ptrs(g, scratch);
   plan_kernel<<<static_cast<unsigned>((ntiles + 127) / 128), 128, 0, s>>>(
       rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, pp.cnt, pp.tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_plan(const sla_block_lists& lists, int BH, int nrb, int ncb, int rb,
+                             int cb, int32_t* cnt, uint32_t* tiles, cudaStream_t s) {
+  const int nt = rb == 128 ? nrb : (nrb + 1) / 2;
+  const size_t ntiles = static_cast<size_t>(BH) * nt;
+  if (ntiles == 0) return cudaSuccess;
+  plan_kernel<<<static_cast<unsigned>((ntiles + 127) / 128), 128, 0, s>>>(lists, BH, nrb, ncb, nt,
+                                                                          rb, cb, cnt, tiles);
   return cudaGetLastError();
 }
 

@@ -58,6 +58,25 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v,
                            float* o_s, float* lse, int32_t* status,
                            void* scratch, cudaStream_t s);
 size_t attn_tc_scratch_bytes(const Geom& g);
+// Tile plan of block lists (the attention kernels' work list): lists of
+// `nrb` blocks of `rb` rows (per bh) over `ncb` blocks of `cb` columns are
+// grouped into 128-row tiles (one block of 128 or two of 64) whose merged,
+// sorted column lists are packed two 16-bit entries per word when cb = 64
+// (one otherwise): bit 15 present, bits 13-14 which of the tile's 64-row
+// halves the entry holds for, bits 0-12 column block.  cnt[BH * nt] words
+// per tile, tiles[BH * nt][ncb], nt = ceil(nrb * rb / 128).
+constexpr uint32_t kPlanPresent = 1u << 15;
+cudaError_t launch_tile_plan(const sla_block_lists& lists, int BH, int nrb, int ncb, int rb,
+                             int cb, int32_t* cnt, uint32_t* tiles, cudaStream_t s);
+
+// backward of the critical branch on the tensor cores (attn_bwd_tc.cu):
+// dq, dk, dv are overwritten (fp32); the linear branch adds to them later.
+size_t attn_bwd_tc_scratch_bytes(const Geom& g);
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* delta,
+                               const sla_block_lists& rows, const sla_block_lists& cols,
+                               float* dq, float* dk, float* dv, const Geom& g, void* scratch,
+                               int32_t* status, cudaStream_t s);
 // Outputs of the fused tensor-core attention; any pointer may be null.
 struct AttnOutputs {
   float* o_s;     // fp32 O_s

@@ -72,7 +72,7 @@ bool has_linear_branch(const Geom& g) { return g.linear; }
 // Workspace layouts (each region 256-byte aligned).
 struct MaskWs { size_t qbar, kbar, logits, total; };
 struct FwdWs { size_t o_s, hsum, zsum, lintc, tc, total; };
-struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, total; };
+struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, plans, total; };
 
 MaskWs mask_ws(const Geom& g) {
   MaskWs w;
@@ -115,6 +115,9 @@ BwdWs bwd_ws(const Geom& g) {
     w.dzm = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d);
   }
   w.dwp = off; off = align_up(off + sizeof(float) * size_t(sla::bwd_dw_parts(g)) * g.d * g.d);
+  w.plans = off;
+  if (g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g))
+    off = align_up(off + sla::attn_bwd_tc_scratch_bytes(g));
   w.total = off;
   return w;
 }
@@ -393,8 +396,13 @@ sla_status sla_backward(const sla_params* p, const void* q, const void* k,
   float* gbuf = at<float>(ws, w.gbuf);
   float* dwp = at<float>(ws, w.dwp);
   SLA_CUDA(sla::launch_bwd_prep(dout, o_s, o_lin, proj, delta, gbuf, dwp, g, s));
-  SLA_CUDA(sla::launch_attn_bwd_dq(q, k, v, dout, lse, delta, *rows, dq, g, s));
-  SLA_CUDA(sla::launch_attn_bwd_dkdv(q, k, v, dout, lse, delta, *cols, dk, dv, g, s));
+  if (g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g)) {
+    SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
+                                     at<char>(ws, w.plans), static_cast<int32_t*>(ws), s));
+  } else {
+    SLA_CUDA(sla::launch_attn_bwd_dq(q, k, v, dout, lse, delta, *rows, dq, g, s));
+    SLA_CUDA(sla::launch_attn_bwd_dkdv(q, k, v, dout, lse, delta, *cols, dk, dv, g, s));
+  }
   if (has_linear_branch(g)) {
     float* hsum = at<float>(ws, w.hsum);
     float* zsum = at<float>(ws, w.zsum);

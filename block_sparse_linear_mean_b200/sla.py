@@ -352,7 +352,7 @@ def backward(p: sla_params, q, k, v, proj, dout, rows: BlockLists, cols: BlockLi
                                         saved["o_lin"].data_ptr(), dq.data_ptr(),
                                         dk.data_ptr(), dv.data_ptr(), dproj.data_ptr(),
                                         ws.data_ptr(), ws.numel(), _stream()))
-    return dict(dq=dq, dk=dk, dv=dv, dproj=dproj)
+    return dict(dq=dq, dk=dk, dv=dv, dproj=dproj, ws=ws)
 
 
 def check_device_status(ws: torch.Tensor) -> int:

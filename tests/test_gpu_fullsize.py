@@ -85,6 +85,7 @@ def test_full_size_backward_one_head_slice():
     f = sla.forward(p, x.q, x.k, x.v, x.proj, m["rows"], save_for_backward=True)
     g = sla.backward(p, x.q, x.k, x.v, x.proj, x.dout, m["rows"], m["cols"], f)
     torch.cuda.synchronize()
+    assert sla.check_device_status(g["ws"]) == sla.SLA_OK
     mask = m["mask"].cpu().numpy()
     o = orc.backward(x.q.cpu(), x.k.cpu(), x.v.cpu(), x.proj.cpu(), mask, x.dout.cpu(),
                      wl.block_q, wl.block_k)

@@ -121,18 +121,23 @@ def test_forward_matches_oracle_with_oracle_mask(case, simt):
     print(name, "simt" if simt else "default", {k: f"{v[0]:.2e}/{v[1]:.2e}" for k, v in res.items()})
 
 
-def test_backward_matches_oracle(case):
+@pytest.mark.parametrize("simt", [False, True], ids=["default", "simt"])
+def test_backward_matches_oracle(case, simt):
     name, wl, x, t, ref = case
-    p = sla.params_from(t["q"], wl)
+    if simt and wl.dtype == "f32":
+        pytest.skip("fp32 always runs the SIMT kernels")
+    p = sla.params_from(t["q"], wl, simt=simt)
     _, rows, cols = feed_mask(p, ref["mask"])
     f = sla.forward(p, t["q"], t["k"], t["v"], t["proj"], rows, save_for_backward=True)
     g = sla.backward(p, t["q"], t["k"], t["v"], t["proj"], t["dout"], rows, cols, f)
     torch.cuda.synchronize()
+    st = sla.check_device_status(g["ws"])
+    assert st == sla.SLA_OK, sla.status_string(st)
     o = orc.backward(x.q, x.k, x.v, x.proj, ref["mask"], x.dout, wl.block_q, wl.block_k)
     res = {}
     for key in ("dq", "dk", "dv", "dproj"):
         res[key] = assert_close(to_np(g[key]), o[key], wl.dtype, f"{name}.{key}", rel=True)
-    print(name, {k: f"{v[0]:.2e}/{v[1]:.2e}" for k, v in res.items()})
+    print(name, "simt" if simt else "default", {k: f"{v[0]:.2e}/{v[1]:.2e}" for k, v in res.items()})
 
 
 # ---------------------------------------------------------------- edge cases
