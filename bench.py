@@ -269,9 +269,17 @@ def run_ours(args, rank, world, local_rank):
     launches_per_step = 4 + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
         + (1 if (not fused and wl.frac_marg > 0) else 0) + (1 if fused else 2)
     if bwd:
-        # column lists | Delta and g, dW partials, dQ, dK dV, (summaries,
-        # linear dq, linear dk dv), dW reduction
-        launches_per_step += 1 + 5 + (3 if wl.frac_marg > 0 else 0)
+        lin = wl.frac_marg > 0
+        launches_per_step += 1  # column lists
+        if fused and wl.d == 128:
+            # Delta | 2 tile plans, dq, dkdv | (W to bf16, summaries,
+            # indicator, gather, linear q side, indicator + gather of dH,
+            # linear kv side, dW partials, dW sum)
+            launches_per_step += 1 + 4 + (10 if lin else 0)
+        else:
+            # Delta and g, dW partials | dq, dkdv (tcgen05: + 2 tile plans) |
+            # (summaries, linear dq, linear dk dv) | dW reduction
+            launches_per_step += 2 + (4 if fused else 2) + (3 if lin else 0) + 1
 
 
     # warm-up (also fixes the mask used to count the algorithmic work)

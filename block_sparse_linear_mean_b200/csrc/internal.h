@@ -117,6 +117,24 @@ cudaError_t launch_lin_tc_prepare(const void* k, const void* v, const float* pro
                                   const sla_block_lists& rows, const Geom& g, void* scratch,
                                   int32_t* status, cudaStream_t s);
 LinInputs lin_tc_inputs(const Geom& g, void* scratch, const sla_block_lists& rows);
+// Indicator GEMM over the marginal part of `lists` (nrow lists over ncol
+// blocks per bh): dst_h[bh][r] = sum of src_h[bh][x] (bf16 d x d) and
+// dst_z[bh][r] = sum of src_z[bh][x] (fp32 d) over x in list r.  `ind` holds
+// BH * nrow * ld bf16 (ld = ncol rounded up to 64).
+cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, int ncol,
+                               const void* src_h, const float* src_z, void* dst_h, float* dst_z,
+                               void* ind, int ld, int32_t* status, cudaStream_t s);
+
+// backward of the linear branch and the projection on the tensor cores
+// (lin_bwd_tc.cu): dq, dk, dv are added to; dproj is written.
+size_t lin_bwd_tc_scratch_bytes(const Geom& g);
+cudaError_t launch_delta(const void* dout, const float* o_s, float* delta, const Geom& g,
+                         cudaStream_t s);
+cudaError_t launch_lin_bwd_tc(const void* q, const void* k, const void* v, const float* proj,
+                              const void* dout, const sla_block_lists& rows,
+                              const sla_block_lists& cols, const float* o_lin, float* dq,
+                              float* dk, float* dv, float* dproj, const Geom& g, void* scratch,
+                              int32_t* status, cudaStream_t s);
 
 // backward
 cudaError_t launch_bwd_prep(const void* dout, const float* o_s,

@@ -494,6 +494,31 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
                                float* o_lin, const Geom& g, void* scratch, int32_t* status,
                                cudaStream_t s, bool prepare, bool apply);
 
+cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, int ncol,
+                               const void* src_h, const float* src_z, void* dst_h, float* dst_z,
+                               void* ind, int ld, int32_t* status, cudaStream_t s) {
+  cudaError_t e;
+  uint16_t* indp = static_cast<uint16_t*>(ind);
+  indicator_kernel<<<BH * nrow, 128, 0, s>>>(lists, indp, src_z, dst_z, nrow, ncol, ld);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  CUtensorMap mA, mB, mC;
+  const uint64_t bh = BH, nr = nrow, nc = ncol, l = ld;
+  const uint64_t da[3] = {l, nr, bh}, sa[2] = {l * 2, nr * l * 2};
+  const uint32_t ba[3] = {64, 128, 1};
+  const uint64_t db[3] = {kHElems, nc, bh}, sbt[2] = {kHElems * 2, nc * kHElems * 2};
+  const uint32_t bb[3] = {64, 64, 1};
+  const uint64_t dc[3] = {kHElems, nr, bh}, sc2[2] = {kHElems * 2, nr * kHElems * 2};
+  const uint32_t bc[3] = {64, 128, 1};
+  if (!encode_bf16_map(&mA, indp, 3, da, sa, ba) || !encode_bf16_map(&mB, src_h, 3, db, sbt, bb) ||
+      !encode_bf16_map(&mC, dst_h, 3, dc, sc2, bc))
+    return cudaErrorInvalidValue;
+  const size_t smem = kGStages * kGStage + 256 + 1024;
+  if ((e = set_smem(gather_gemm_kernel, smem)) != cudaSuccess) return e;
+  dim3 grid(kHElems / 256, (nrow + 127) / 128, BH);
+  gather_gemm_kernel<<<grid, 192, smem, s>>>(mA, mB, mC, ld / 64, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_lin_tc_prepare(const void* k, const void* v, const float* proj,
                                   const sla_block_lists& rows, const Geom& g, void* scratch,
                                   int32_t* status, cudaStream_t s) {

@@ -72,7 +72,15 @@ bool has_linear_branch(const Geom& g) { return g.linear; }
 // Workspace layouts (each region 256-byte aligned).
 struct MaskWs { size_t qbar, kbar, logits, total; };
 struct FwdWs { size_t o_s, hsum, zsum, lintc, tc, total; };
-struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, plans, total; };
+struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, plans, lin, total; };
+
+// Which backward kernels run: the tcgen05 attention backward for bf16
+// (unless SLA_FLAG_SIMT), and with it the tcgen05 linear-branch and
+// projection backward when d = 128; SIMT fp32 kernels otherwise.
+bool bwd_tc_attention(const Geom& g) {
+  return g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g);
+}
+bool bwd_tc_linear(const Geom& g) { return bwd_tc_attention(g) && sla::lin_tc_supported(g); }
 
 MaskWs mask_ws(const Geom& g) {
   MaskWs w;
@@ -106,6 +114,14 @@ BwdWs bwd_ws(const Geom& g) {
   BwdWs w;
   size_t off = kStatusBytes;
   w.delta = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.N);
+  if (bwd_tc_linear(g)) {  // everything else lives in the tensor-core scratch
+    w.gbuf = w.hsum = w.zsum = w.dhm = w.dzm = w.dwp = off;
+    w.plans = off; off = align_up(off + sla::attn_bwd_tc_scratch_bytes(g));
+    w.lin = off; off = align_up(off + sla::lin_bwd_tc_scratch_bytes(g));
+    w.total = off;
+    return w;
+  }
+  w.lin = off;
   w.gbuf = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.N * g.d);
   w.hsum = w.zsum = w.dhm = w.dzm = off;
   if (has_linear_branch(g)) {
@@ -116,8 +132,7 @@ BwdWs bwd_ws(const Geom& g) {
   }
   w.dwp = off; off = align_up(off + sizeof(float) * size_t(sla::bwd_dw_parts(g)) * g.d * g.d);
   w.plans = off;
-  if (g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g))
-    off = align_up(off + sla::attn_bwd_tc_scratch_bytes(g));
+  if (bwd_tc_attention(g)) off = align_up(off + sla::attn_bwd_tc_scratch_bytes(g));
   w.total = off;
   return w;
 }
@@ -393,10 +408,19 @@ sla_status sla_backward(const sla_params* p, const void* q, const void* k,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
   float* delta = at<float>(ws, w.delta);
+  int32_t* status = static_cast<int32_t*>(ws);
+  if (bwd_tc_linear(g)) {
+    SLA_CUDA(sla::launch_delta(dout, o_s, delta, g, s));
+    SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
+                                     at<char>(ws, w.plans), status, s));
+    SLA_CUDA(sla::launch_lin_bwd_tc(q, k, v, proj, dout, *rows, *cols, o_lin, dq, dk, dv, dproj, g,
+                                    at<char>(ws, w.lin), status, s));
+    return SLA_OK;
+  }
   float* gbuf = at<float>(ws, w.gbuf);
   float* dwp = at<float>(ws, w.dwp);
   SLA_CUDA(sla::launch_bwd_prep(dout, o_s, o_lin, proj, delta, gbuf, dwp, g, s));
-  if (g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g)) {
+  if (bwd_tc_attention(g)) {
     SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
                                      at<char>(ws, w.plans), static_cast<int32_t*>(ws), s));
   } else {
