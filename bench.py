@@ -46,9 +46,12 @@ L2_BYTES = 126 * 1024 * 1024
 # lanes x 2 flops x 1.965 GHz (max SM clock).
 FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes per launch of the dominant kernel from an ncu capture of the
-# current kernel version (None until captured for that version).
-TRAFFIC_PER_LAUNCH = {}
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of the current kernel version (dram__bytes_read.sum +
+# dram__bytes_write.sum; command and figures in profiles/); absent = null.
+TRAFFIC_PER_LAUNCH = {
+    ("sla_1p3b", "attn_tc"): 506_972_416 + 90_471_936,  # profiles/attn_tc_sla_1p3b.md
+}
 
 
 def parse():
@@ -149,18 +152,27 @@ class ClockSampler:
         self.err = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
 
+    def _sample_once(self):
+        import pynvml as nv
+        try:
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+            self.samples.append((time.time(), sm, rs, pw))
+        except Exception as e:  # keep sampling; record the last error
+            self.err = repr(e)
+
     def _run(self):
         import pynvml as nv
-        h = nv.nvmlDeviceGetHandleByIndex(self.idx)
-        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        try:
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception as e:
+            self.err = repr(e)
+            return
         while not self._stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((time.time(), sm, rs, pw))
-            except Exception as e:  # keep sampling; record the last error
-                self.err = repr(e)
+            self._sample_once()
             self._stop.wait(self.period)
 
     def __enter__(self):
@@ -172,12 +184,17 @@ class ClockSampler:
             nv.nvmlInit()
             self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
+            # the timed region starts only once sampling runs
+            t0 = time.time()
+            while not self.samples and self.err is None and time.time() - t0 < 5.0:
+                time.sleep(0.001)
         except Exception as e:
             self.err = repr(e)
         return self
 
     def __exit__(self, *exc):
         if self.thread is not None:
+            self._sample_once()  # one sample at the end of the timed region
             self._stop.set()
             self.thread.join(timeout=5)
         try:
@@ -455,7 +472,7 @@ def blas_threads():
 
 
 def cpu_baseline(wl):
-    heads, flops, secs = oracle_sample(wl, heads=min(wl.H, 4), min_seconds=10.0)
+    heads, flops, secs = oracle_sample(wl, heads=wl.H, min_seconds=12.0)
     return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
             "kind": "oracle",
             "sample": f"float64 oracle mask + forward on {heads} of {wl.H} heads "
