@@ -550,15 +550,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
     // all P V products done: O final in TMEM, Q, the K/V stages and the S
     // columns free
+    // linear branch: this thread's half row of z^M (channels [64h, 64h + 64)),
+    // fetched in one batch while the last P V products finish
+    const bool second = BQ == 64 && r >= 64;
+    const int nm_r = second ? nm_b : nm_a;
+    float4 z4[16];
+    if (D == 128 && lin && nm_r > 0) {
+      const float4* zp = reinterpret_cast<const float4*>(
+          ep.zm + (i64(bh) * nqb + (second ? qb2 : qa)) * 128 + h * 64);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z4[i] = __ldg(zp + i);
+    }
     if (fin && T > 0) fin = __all_sync(full, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
     bool lin_ok = false;
     if (D == 128 && lin && fin) {  // (never taken for d = 64: lin is false)
       // phi(Q) in place (this thread: row r, channels [64h, 64h + 64)), and
       // half of the normaliser phi(q) . z^M from the same rounded values
-      const bool second = BQ == 64 && r >= 64;
-      const int nm_r = second ? nm_b : nm_a;
-      const float* zrow = ep.zm + (i64(bh) * nqb + (second ? qb2 : qa)) * 128 + h * 64;
-      float dpart = 0.f;
+      float dpart = 0.f, dpart2 = 0.f;
       lin_ok = __all_sync(full, wait(b_q, 0));
       if (lin_ok) {
 #pragma unroll
@@ -567,16 +575,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           uint4 val = make_uint4(0u, 0u, 0u, 0u);
           if (row < N && nm_r > 0) {
             val = phi_unit(*p);
-            const uint32_t w4[4] = {val.x, val.y, val.z, val.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-              dpart = fmaf(f.x, __ldg(zrow + u * 8 + 2 * e), dpart);
-              dpart = fmaf(f.y, __ldg(zrow + u * 8 + 2 * e + 1), dpart);
-            }
+            const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.x));
+            const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.y));
+            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.z));
+            const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.w));
+            const float4 za = z4[2 * u], zb = z4[2 * u + 1];
+            dpart = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, fmaf(f1.y, za.w, dpart))));
+            dpart2 = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, dpart2))));
           }
           *p = val;
         }
+        dpart += dpart2;
         const int db = fb ^ 1;  // slot of tile T-1, read by all before b_fin
         red[(db * 2 + h) * 128 + r] = dpart;
         fence_async_smem();
