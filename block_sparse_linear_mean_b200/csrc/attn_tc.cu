@@ -39,6 +39,7 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 3;
+constexpr int kSBuf = 3;  // S tiles in TMEM (P of a tile overwrites its S)
 // One pair in kPolyEvery of a full tile's exponentials is computed by a cubic
 // on the FMA pipe instead of the special-function unit (0: none).
 constexpr int kPolyEvery = 3;
@@ -153,33 +154,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t sb = raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
   constexpr int kB0 = 1 + 4 * kStages;            // first barrier after the K/V rings
-  static_assert((kB0 + 28) * 8 <= kUsed - offBar, "barrier block too small");
   const uint32_t b_q = smem_u32(&bars[0]);
   auto b_k_full = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto b_v_full = [&](int s) { return smem_u32(&bars[1 + kStages + s]); };
   auto b_k_empty = [&](int s) { return smem_u32(&bars[1 + 2 * kStages + s]); };
   auto b_v_empty = [&](int s) { return smem_u32(&bars[1 + 3 * kStages + s]); };
-  auto b_s_full = [&](int b) { return smem_u32(&bars[kB0 + b]); };
-  auto b_s_free = [&](int b) { return smem_u32(&bars[kB0 + 2 + b]); };
-  auto b_p_full = [&](int b) { return smem_u32(&bars[kB0 + 4 + b]); };
-  auto b_pv_done = [&](int b) { return smem_u32(&bars[kB0 + 6 + b]); };
+  // per S buffer j = t % kSBuf: S(t) in TMEM, P(t) in TMEM (8 warps), P V of
+  // tile t done
+  auto b_s_full = [&](int j) { return smem_u32(&bars[kB0 + j]); };
+  auto b_p_full = [&](int j) { return smem_u32(&bars[kB0 + kSBuf + j]); };
+  auto b_pv_done = [&](int j) { return smem_u32(&bars[kB0 + 2 * kSBuf + j]); };
+  constexpr int kB1 = kB0 + 3 * kSBuf;
   // partial row maxima exchanged between the two warps holding the same 32
   // rows (one per column half): one barrier per (tile parity, lane quadrant)
-  auto b_red = [&](int b, int quad) { return smem_u32(&bars[kB0 + 18 + 4 * b + quad]); };
-  const uint32_t b_fin = smem_u32(&bars[kB0 + 10]);
-  const uint32_t b_lin = smem_u32(&bars[kB0 + 11]);   // H^M and W tiles landed
-  const uint32_t b_phiq = smem_u32(&bars[kB0 + 12]);  // phi(Q) written (8 warps)
-  const uint32_t b_den = smem_u32(&bars[kB0 + 13]);   // normaliser halves exchanged (8 warps)
-  const uint32_t b_num = smem_u32(&bars[kB0 + 14]);   // phi(Q) H^M in TMEM
-  const uint32_t b_olin = smem_u32(&bars[kB0 + 15]);  // O_lin (bf16) in shared memory (8 warps)
-  const uint32_t b_lout = smem_u32(&bars[kB0 + 16]);  // O_lin W in TMEM
+  auto b_red = [&](int b, int quad) { return smem_u32(&bars[kB1 + 9 + 4 * b + quad]); };
+  const uint32_t b_fin = smem_u32(&bars[kB1 + 0]);
+  const uint32_t b_lin = smem_u32(&bars[kB1 + 1]);   // H^M and W tiles landed
+  const uint32_t b_phiq = smem_u32(&bars[kB1 + 2]);  // phi(Q) written (8 warps)
+  const uint32_t b_den = smem_u32(&bars[kB1 + 3]);   // normaliser halves exchanged (8 warps)
+  const uint32_t b_num = smem_u32(&bars[kB1 + 4]);   // phi(Q) H^M in TMEM
+  const uint32_t b_olin = smem_u32(&bars[kB1 + 5]);  // O_lin (bf16) in shared memory (8 warps)
+  const uint32_t b_lout = smem_u32(&bars[kB1 + 6]);  // O_lin W in TMEM
   // every P V product done (single use).  The producer cannot wait on
-  // pv_done for this: with more than two stages the completion before the
-  // last one on the same barrier may still be pending, and a parity wait
-  // would then take the older phase for the newer one.
-  const uint32_t b_pv_last = smem_u32(&bars[kB0 + 17]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB0 + 26]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB0 + 27]);
+  // pv_done for this: the completion before the last one on the same
+  // barrier may still be pending, and a parity wait would then take the
+  // older phase for the newer one.
+  const uint32_t b_pv_last = smem_u32(&bars[kB1 + 7]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB1 + 17]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB1 + 18]);
+  static_assert((kB1 + 19) * 8 <= kUsed - offBar, "barrier block too small");
   float* red = reinterpret_cast<float*>(base + offRed);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -214,13 +217,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(b_k_empty(s), 1);
       mbar_init(b_v_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(b_s_full(b), 1);
-      mbar_init(b_s_free(b), kSoftmaxWarps);
-      mbar_init(b_p_full(b), kSoftmaxWarps);
-      mbar_init(b_pv_done(b), 1);
-      for (int q = 0; q < 4; ++q) mbar_init(b_red(b, q), 2);
+    for (int j = 0; j < kSBuf; ++j) {
+      mbar_init(b_s_full(j), 1);
+      mbar_init(b_p_full(j), kSoftmaxWarps);
+      mbar_init(b_pv_done(j), 1);
     }
+    for (int b = 0; b < 2; ++b)
+      for (int q = 0; q < 4; ++q) mbar_init(b_red(b, q), 2);
     mbar_init(b_fin, kSoftmaxWarps);
     mbar_init(b_lin, 1);
     mbar_init(b_phiq, kSoftmaxWarps);
@@ -232,7 +235,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // TMEM: 512 columns (S0 | S1 | O)
+  if (warp == 1) {  // TMEM: 512 columns (S0 | S1 | S2 | O)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -241,12 +244,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // columns: S of tiles with parity b at 128 b, O at 256, bf16 P of parity b
-  // (two keys per column) at 384 + 64 b.  Computed, not indexed from an
-  // array, so no address goes through local memory.
-  auto tS = [&](int b) { return tmem + 128u * static_cast<uint32_t>(b); };
-  const uint32_t tO = tmem + 256;
-  auto tP = [&](int b) { return tmem + 384u + 64u * static_cast<uint32_t>(b); };
+  // columns: S of tile t at 128 (t % kSBuf), O at 384.  The bf16 P of tile t
+  // (two keys per column) overwrites its own S: the column half h puts its
+  // 32 P columns at 64 h, columns that only its own threads read.
+  // Addresses are computed, not indexed from an array, so none goes through
+  // local memory.
+  auto tS = [&](int j) { return tmem + 128u * static_cast<uint32_t>(j); };
+  const uint32_t tO = tmem + 384;
 
   auto give_up = [&]() {
     *abort_flag = 1;
@@ -331,39 +335,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0 && T > 0) {
       bool ok = wait(b_q, 0);
       auto issue_s = [&](int t) -> bool {
-        const int s = t % kStages, b = t & 1;
+        const int s = t % kStages, j = t % kSBuf;
         if (!wait(b_k_full(s), (t / kStages) & 1)) return false;
-        if (t >= 2 && !wait(b_s_free(b), ((t >> 1) & 1) ^ 1)) return false;
+        // S(t) takes the buffer of tile t - kSBuf: that tile's softmax is done
+        // (its P V was issued after its P arrived) and the tensor pipe reads
+        // that P before this MMA overwrites it (it runs in issue order)
         tc_fence_after();
         const uint32_t kbase = sb + offK + s * kKBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          tc_mma(tS(b), sdesc(sb + offQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), idesc_qk,
+          tc_mma(tS(j), sdesc(sb + offQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), idesc_qk,
                  kk > 0);
         }
-        tc_commit(b_s_full(b));
+        tc_commit(b_s_full(j));
         tc_commit(b_k_empty(s));
         return true;
       };
       auto issue_pv = [&](int t) -> bool {
-        const int s = t % kStages, b = t & 1;
-        if (!wait(b_p_full(b), (t >> 1) & 1)) return false;
+        const int s = t % kStages, j = t % kSBuf;
+        if (!wait(b_p_full(j), (t / kSBuf) & 1)) return false;
         if (!wait(b_v_full(s), (t / kStages) & 1)) return false;
         tc_fence_after();
         const uint32_t vbase = sb + offV + s * kKBytes;
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
-          tc_mma_ts(tO, tP(b) + kk * 8, sdesc(vbase + kk * 2048, 16384, 1024), idesc_pv,
-                    (t > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tO, tS(j) + 64 * (kk / 4) + (kk % 4) * 8, sdesc(vbase + kk * 2048, 16384, 1024),
+                    idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(b_v_empty(s));
-        tc_commit(b_pv_done(b));
+        tc_commit(b_pv_done(j));
         return true;
       };
+      // S runs two tiles ahead of P V, so a softmax warp that finishes tile
+      // t finds S(t + 1) computed even when other warps are still on t
       if (ok) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
-        if (t + 1 < T) ok = issue_s(t + 1);
-        if (ok) ok = issue_pv(t);
+        ok = issue_pv(t);
+        if (ok && t + 2 < T) ok = issue_s(t + 2);
       }
       if (ok) tc_commit(b_pv_last);
     }
@@ -414,7 +423,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; ok && t < T; ++t) {
-      const int b = t & 1;
+      const int b = t & 1, j = t % kSBuf;
       const uint32_t desc = ptiles[t];
       // this thread's 64 keys: entry h of a tile of two 64-blocks, or half h
       // of one 128-block
@@ -422,16 +431,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int blk = ent & 0x1FFF;
       const bool member = (ent & kPresent) && (((ent >> 13) & 3u) & rflag);
       const int kvalid = member ? max(0, min(64, N - blk * BK - (BK == 128 ? h * 64 : 0))) : 0;
-      if (!__all_sync(full, wait(b_s_full(b), (t >> 1) & 1))) { ok = false; break; }
+      if (!__all_sync(full, wait(b_s_full(j), (t / kSBuf) & 1))) { ok = false; break; }
       tc_fence_after();
       float s[64];
-      tmem_ld32(tS(b) + lane_off + h * 64, s);
-      tmem_ld32(tS(b) + lane_off + h * 64 + 32, s + 32);
+      tmem_ld32(tS(j) + lane_off + h * 64, s);
+      tmem_ld32(tS(j) + lane_off + h * 64 + 32, s + 32);
       tmem_wait_ld();
       reg_fence<64>(s);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_s_free(b));
       // partial max of the raw scores over this thread's valid keys (four
       // independent three-input chains)
       float mx = -INFINITY;
@@ -506,18 +512,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       acc0 = add2(add2(acc0, acc1), add2(acc2, acc3));
       l += acc0.x + acc0.y;
-      // P buffer b is free once P V of tile t-2 completed
-      if (t >= 2 && !__all_sync(full, wait(b_pv_done(b), ((t >> 1) & 1) ^ 1))) {
-        ok = false;
-        break;
-      }
-      // P (bf16 pairs) into TMEM: this half's 64 keys are columns [32h, 32h + 32)
-      tc_fence_after();
-      tmem_st32u(tP(b) + lane_off + h * 32, pk);
+      // P (bf16 pairs) over this half's own S columns: its 64 keys become
+      // columns [64h, 64h + 32) of the tile's buffer
+      tmem_st32u(tS(j) + lane_off + h * 64, pk);
       // rescale this half of O (warp-wide TMEM access) once the previous
-      // P V is complete
+      // P V is complete.  That parity wait cannot mistake an older phase:
+      // S(t) has completed and was issued after P V of tile t - 2, so P V of
+      // tile t - 4 (the barrier's previous use) is complete.
       if (__any_sync(full, rescale)) {
-        if (t >= 1 && !__all_sync(full, wait(b_pv_done((t - 1) & 1), ((t - 1) >> 1) & 1))) {
+        if (t >= 1 && !__all_sync(full, wait(b_pv_done((t - 1) % kSBuf), ((t - 1) / kSBuf) & 1))) {
           ok = false;
           break;
         }
@@ -536,7 +539,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_st();  // P (and any rescaled O) stored
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_p_full(b));
+      if (lane == 0) mbar_arrive(b_p_full(j));
     }
     // epilogue: total row sum from both halves, O / l, LSE
     const int fb = T & 1;  // red slot last used by tile T-2, read by all
@@ -561,7 +564,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int i = 0; i < 16; ++i) z4[i] = __ldg(zp + i);
     }
-    if (fin && T > 0) fin = __all_sync(full, wait(b_pv_done((T - 1) & 1), ((T - 1) >> 1) & 1));
+    if (fin && T > 0)
+      fin = __all_sync(full, wait(b_pv_done((T - 1) % kSBuf), ((T - 1) / kSBuf) & 1));
     bool lin_ok = false;
     if (D == 128 && lin && fin) {  // (never taken for d = 64: lin is false)
       // phi(Q) in place (this thread: row r, channels [64h, 64h + 64)), and
