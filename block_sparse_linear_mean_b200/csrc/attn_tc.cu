@@ -334,19 +334,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && T > 0) {
       bool ok = wait(b_q, 0);
+      // base descriptors, built once; each MMA advances one by a constant
+      const uint64_t dQ = sdesc(sb + offQ, 16, 1024);
+      const uint64_t dK0 = sdesc(sb + offK, 16, 1024);
+      const uint64_t dV0 = sdesc(sb + offV, 16384, 1024);
       auto issue_s = [&](int t) -> bool {
         const int s = t % kStages, j = t % kSBuf;
         if (!wait(b_k_full(s), (t / kStages) & 1)) return false;
         // S(t) takes the buffer of tile t - kSBuf: that tile's softmax is done
-        // (its P V was issued after its P arrived) and the tensor pipe reads
-        // that P before this MMA overwrites it (it runs in issue order)
+        // (its P V was issued after its P arrived, before this call) and the
+        // tensor pipe reads that P before this MMA overwrites it (it runs in
+        // issue order)
         tc_fence_after();
-        const uint32_t kbase = sb + offK + s * kKBytes;
+        const uint64_t dK = sdesc_add(dK0, s * kKBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          tc_mma(tS(j), sdesc(sb + offQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), idesc_qk,
-                 kk > 0);
+          tc_mma(tS(j), sdesc_add(dQ, off), sdesc_add(dK, off), idesc_qk, kk > 0);
         }
         tc_commit(b_s_full(j));
         tc_commit(b_k_empty(s));
@@ -357,22 +361,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!wait(b_p_full(j), (t / kSBuf) & 1)) return false;
         if (!wait(b_v_full(s), (t / kStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t vbase = sb + offV + s * kKBytes;
+        const uint64_t dV = sdesc_add(dV0, s * kKBytes);
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
-          tc_mma_ts(tO, tS(j) + 64 * (kk / 4) + (kk % 4) * 8, sdesc(vbase + kk * 2048, 16384, 1024),
-                    idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tO, tS(j) + 64 * (kk / 4) + (kk % 4) * 8, sdesc_add(dV, kk * 2048), idesc_pv,
+                    (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(b_v_empty(s));
         tc_commit(b_pv_done(j));
         return true;
       };
-      // S runs two tiles ahead of P V, so a softmax warp that finishes tile
-      // t finds S(t + 1) computed even when other warps are still on t
+      // S(t + 2) is issued before the wait for P(t) (its buffer was last
+      // read by P V of tile t - 1, issued in the previous round), so the
+      // tensor pipe computes it while the softmax works on tile t, and a
+      // softmax warp that finishes a tile finds the next S already done
       if (ok) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
-        ok = issue_pv(t);
-        if (ok && t + 2 < T) ok = issue_s(t + 2);
+        if (t + 2 < T) ok = issue_s(t + 2);
+        if (ok) ok = issue_pv(t);
       }
       if (ok) tc_commit(b_pv_last);
     }
@@ -422,9 +428,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const unsigned full = 0xffffffffu;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    // the plan word of the next tile is fetched a tile ahead: a global load
+    // on the path from one tile to the next would stall every warp
+    uint32_t desc_next = T > 0 ? ptiles[0] : 0u;
     for (int t = 0; ok && t < T; ++t) {
       const int b = t & 1, j = t % kSBuf;
-      const uint32_t desc = ptiles[t];
+      const uint32_t desc = desc_next;
+      if (t + 1 < T) desc_next = ptiles[t + 1];
       // this thread's 64 keys: entry h of a tile of two 64-blocks, or half h
       // of one 128-block
       const uint32_t ent = BK == 64 ? (desc >> (16 * h)) & 0xFFFFu : desc & 0xFFFFu;
@@ -517,7 +527,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_st32u(tS(j) + lane_off + h * 64, pk);
       // rescale this half of O (warp-wide TMEM access) once the previous
       // P V is complete.  That parity wait cannot mistake an older phase:
-      // S(t) has completed and was issued after P V of tile t - 2, so P V of
+      // S(t) has completed and was issued after P V of tile t - 3, so P V of
       // tile t - 4 (the barrier's previous use) is complete.
       if (__any_sync(full, rescale)) {
         if (t >= 1 && !__all_sync(full, wait(b_pv_done((t - 1) % kSBuf), ((t - 1) / kSBuf) & 1))) {

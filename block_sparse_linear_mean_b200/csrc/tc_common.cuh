@@ -226,6 +226,16 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// A descriptor advanced by `bytes` (a multiple of 16): the start address
+// field holds address / 16 in its low 14 bits, and shared addresses stay
+// below 256 KB, so the add never carries out of the field.  Building each
+// base descriptor once and advancing it this way keeps the per-MMA issue
+// cost to one 64-bit add; rebuilding a descriptor per MMA costs the issuing
+// thread more than the MMA itself takes on the tensor core.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
 // 1; addresses and byte offsets are encoded in 16-byte units.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
