@@ -206,23 +206,25 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   } else if (warp == 1) {
     if (lane == 0 && U > 0) {
       bool ok = bwait(sh, b_q, 0);
+      // base descriptors, built once and advanced by constant offsets
+      const uint64_t dQd = sdesc(sb + offQ, 16, 1024), ddO = sdesc(sb + offdO, 16, 1024);
+      const uint64_t dKV = sdesc(sb + offKV, 16, 1024), dKVmn = sdesc(sb + offKV, 8192, 1024);
       auto issue_sdp = [&](int u) -> bool {
         const int s = u % kBwdStages, b = u & 1;
         if (!bwait(sh, b_full(s), (u / kBwdStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t kb = sb + offKV + s * kStageBytes;
+        const uint64_t dK = sdesc_add(dKV, s * kStageBytes), dV = sdesc_add(dK, kHalfBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t ob = (kk / 4) * 8192 + (kk % 4) * 32;
-          tc_mma(tS(b), sdesc(sb + offQ + oa, 16, 1024), sdesc(kb + ob, 16, 1024), idesc_s, kk > 0);
+          tc_mma(tS(b), sdesc_add(dQd, oa), sdesc_add(dK, ob), idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t ob = (kk / 4) * 8192 + (kk % 4) * 32;
-          tc_mma(tP(b), sdesc(sb + offdO + oa, 16, 1024), sdesc(kb + kHalfBytes + ob, 16, 1024),
-                 idesc_s, kk > 0);
+          tc_mma(tP(b), sdesc_add(ddO, oa), sdesc_add(dV, ob), idesc_s, kk > 0);
         }
         tc_commit(b_s(b));
         return true;
@@ -231,11 +233,11 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         const int s = u % kBwdStages, b = u & 1;
         if (!bwait(sh, b_ds(b), (u >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t kb = sb + offKV + s * kStageBytes;
+        const uint64_t dKmn = sdesc_add(dKVmn, s * kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 16 keys = 8 columns of dS
-          tc_mma_ts(tQ, tS(b) + 32 * (kk / 2) + (kk % 2) * 8, sdesc(kb + kk * 2048, 8192, 1024),
-                    idesc_dq, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tQ, tS(b) + 32 * (kk / 2) + (kk % 2) * 8, sdesc_add(dKmn, kk * 2048), idesc_dq,
+                    (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit(b_empty(s));
         return true;
       };
@@ -466,23 +468,25 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   } else if (warp == 1) {
     if (lane == 0 && U > 0) {
       bool ok = bwait(sh, b_kv, 0);
+      // base descriptors, built once and advanced by constant offsets
+      const uint64_t dKd = sdesc(sb + offK, 16, 1024), dVd = sdesc(sb + offV, 16, 1024);
+      const uint64_t dSt = sdesc(sb + offSt, 16, 1024), dStmn = sdesc(sb + offSt, 8192, 1024);
       auto issue_sdp = [&](int u) -> bool {
         const int s = u % kBwdStages, b = u & 1;
         if (!bwait(sh, b_full(s), (u / kBwdStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t qb = sb + offSt + s * kStageBytes;
+        const uint64_t dQs = sdesc_add(dSt, s * kStageBytes), ddOs = sdesc_add(dQs, kHalfBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t ob = (kk / 4) * 8192 + (kk % 4) * 32;
-          tc_mma(tS(b), sdesc(sb + offK + oa, 16, 1024), sdesc(qb + ob, 16, 1024), idesc_s, kk > 0);
+          tc_mma(tS(b), sdesc_add(dKd, oa), sdesc_add(dQs, ob), idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t ob = (kk / 4) * 8192 + (kk % 4) * 32;
-          tc_mma(tP(b), sdesc(sb + offV + oa, 16, 1024), sdesc(qb + kHalfBytes + ob, 16, 1024),
-                 idesc_s, kk > 0);
+          tc_mma(tP(b), sdesc_add(dVd, oa), sdesc_add(ddOs, ob), idesc_s, kk > 0);
         }
         tc_commit(b_s(b));
         return true;
@@ -491,16 +495,15 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         const int s = u % kBwdStages, b = u & 1;
         if (!bwait(sh, b_pd(b), (u >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t qb = sb + offSt + s * kStageBytes;
+        const uint64_t dQmn = sdesc_add(dStmn, s * kStageBytes), ddOmn = sdesc_add(dQmn, kHalfBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO: 16 queries = 8 columns
-          tc_mma_ts(tV, tS(b) + 32 * (kk / 2) + (kk % 2) * 8,
-                    sdesc(qb + kHalfBytes + kk * 2048, 8192, 1024), idesc_g,
+          tc_mma_ts(tV, tS(b) + 32 * (kk / 2) + (kk % 2) * 8, sdesc_add(ddOmn, kk * 2048), idesc_g,
                     (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-          tc_mma_ts(tK, tP(b) + 32 * (kk / 2) + (kk % 2) * 8, sdesc(qb + kk * 2048, 8192, 1024),
-                    idesc_g, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tK, tP(b) + 32 * (kk / 2) + (kk % 2) * 8, sdesc_add(dQmn, kk * 2048), idesc_g,
+                    (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit(b_empty(s));
         return true;
       };

@@ -224,15 +224,16 @@ __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16(128, 256, 0, 1);
+    const uint64_t dA = sdesc(sb, 16, 1024), dB = sdesc(sb + kGA, 8192, 1024);  // built once
     for (int ks = 0; ks < ksteps && ok; ++ks) {
       const int s = ks % kGStages;
       ok = wait_bounded(b_full(s), (ks / kGStages) & 1, status, kTimeout);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t st = sb + s * kGStage;
+      const uint32_t so = s * kGStage;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        tc_mma(tmem, sdesc(st + kk * 32, 16, 1024), sdesc(st + kGA + kk * 2048, 8192, 1024), idesc,
+        tc_mma(tmem, sdesc_add(dA, so + kk * 32), sdesc_add(dB, so + kk * 2048), idesc,
                (ks > 0 || kk > 0) ? 1u : 0u);
       tc_commit(b_empty(s));
     }
