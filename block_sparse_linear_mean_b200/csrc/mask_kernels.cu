@@ -126,8 +126,9 @@ cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
 // ---------------------------------------------------------------------------
 // Block-wide helpers (256 threads).
 
-constexpr int kCT = 256;  // classifier threads per CTA
+constexpr int kCT = 256;  // threads per CTA of the list-from-mask kernel
 
+template <int CT>
 __device__ __forceinline__ float block_reduce_max(float v, float* red) {
   v = warp_max(v);
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
@@ -135,10 +136,11 @@ __device__ __forceinline__ float block_reduce_max(float v, float* red) {
   if (l == 0) red[w] = v;
   __syncthreads();
   float r = red[0];
-  for (int i = 1; i < kCT / 32; ++i) r = fmaxf(r, red[i]);
+  for (int i = 1; i < CT / 32; ++i) r = fmaxf(r, red[i]);
   return r;
 }
 
+template <int CT>
 __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
   v = warp_sum(v);
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
@@ -146,10 +148,11 @@ __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
   if (l == 0) red[w] = v;
   __syncthreads();
   float r = red[0];
-  for (int i = 1; i < kCT / 32; ++i) r += red[i];
+  for (int i = 1; i < CT / 32; ++i) r += red[i];
   return r;
 }
 
+template <int CT>
 __device__ __forceinline__ int block_reduce_sum_int(int v, int* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -158,18 +161,19 @@ __device__ __forceinline__ int block_reduce_sum_int(int v, int* red) {
   if (l == 0) red[w] = v;
   __syncthreads();
   int r = 0;
-  for (int i = 0; i < kCT / 32; ++i) r += red[i];
+  for (int i = 0; i < CT / 32; ++i) r += red[i];
   return r;
 }
 
 // Writes the ascending lists of label-2 and label-1 blocks of one row.
 // `lab` (shared) holds n labels; `idx_c`/`idx_m` are the row's list slots.
+template <int CT>
 __device__ void compact_row(const int8_t* lab, int n, int32_t* idx_c,
                             int32_t* cnt_c, int32_t* idx_m, int32_t* cnt_m,
                             int* wsum) {
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
   int base_c = 0, base_m = 0;
-  for (int j0 = 0; j0 < n; j0 += kCT) {
+  for (int j0 = 0; j0 < n; j0 += CT) {
     const int j = j0 + threadIdx.x;
     const int8_t lb = j < n ? lab[j] : 0;
     const unsigned bc = __ballot_sync(0xffffffffu, lb == 2);
@@ -178,7 +182,7 @@ __device__ void compact_row(const int8_t* lab, int n, int32_t* idx_c,
     if (l == 0) { wsum[w] = __popc(bc); wsum[8 + w] = __popc(bm); }
     __syncthreads();
     int off_c = base_c, off_m = base_m, tot_c = 0, tot_m = 0;
-    for (int i = 0; i < kCT / 32; ++i) {
+    for (int i = 0; i < CT / 32; ++i) {
       if (i < w) { off_c += wsum[i]; off_m += wsum[8 + i]; }
       tot_c += wsum[i]; tot_m += wsum[8 + i];
     }
@@ -195,7 +199,8 @@ __device__ void compact_row(const int8_t* lab, int n, int32_t* idx_c,
 }
 
 // ---------------------------------------------------------------------------
-// Classifier: one CTA (256 threads) per (bh, query block) row.
+// Classifier: one CTA per (bh, query block) row (64 threads for rows of up to
+// 1024 blocks, 256 above).
 //   1. P = softmax of the row's logits (fp32, fixed reduction order), kept as
 //      32-bit patterns: scores are non-negative, so the patterns order like
 //      the values;
@@ -224,9 +229,10 @@ __device__ __forceinline__ uint64_t to_fixed(uint32_t pbits) {
   return __double2ull_rz(static_cast<double>(__uint_as_float(pbits)) * kFixedOne);
 }
 
+template <int CT>
 struct SelShared {
-  uint32_t hist[8][256];
-  unsigned long long hsum[8][256];
+  uint32_t hist[(CT / 32)][256];
+  unsigned long long hsum[(CT / 32)][256];
   uint32_t tot[256];
   unsigned long long tots[256];
   uint32_t res_u[4];
@@ -235,24 +241,39 @@ struct SelShared {
 
 // Rank-k score (k counted from the top, 0-based) among the n patterns: the
 // value v and the number of patterns strictly above it.
-__device__ void select_rank(const uint32_t* pb, int n, int k, SelShared& sh, uint32_t& v,
+template <int CT>
+__device__ void select_rank(const uint32_t* pb, int n, int k, SelShared<CT>& sh, uint32_t& v,
                             int& above) {
   const int tid = threadIdx.x, w = tid / 32, lane = tid % 32;
   uint32_t prefix = 0, mask = 0;
   int krem = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 8 * 256; b += kCT) (&sh.hist[0][0])[b] = 0u;
+    for (int b = tid; b < (CT / 32) * 256; b += CT) (&sh.hist[0][0])[b] = 0u;
     __syncthreads();
-    for (int j = tid; j < n; j += kCT) {
-      const uint32_t x = pb[j];
-      if ((x & mask) == prefix) atomicAdd(&sh.hist[w][(x >> shift) & 255u], 1u);
+    if constexpr (CT <= 64) {
+      // few histograms: lanes with equal digits add once, through their
+      // lowest lane (a row's scores share their leading bits, so plain
+      // atomics would collide)
+      for (int j0 = 0; j0 < n; j0 += CT) {
+        const int j = j0 + tid;
+        const uint32_t x = j < n ? pb[j] : 0u;
+        const bool in = j < n && (x & mask) == prefix;
+        const uint32_t dg = in ? (x >> shift) & 255u : 256u;
+        const unsigned peers = __match_any_sync(0xffffffffu, dg);
+        if (in && (lane == __ffs(peers) - 1)) atomicAdd(&sh.hist[w][dg], static_cast<uint32_t>(__popc(peers)));
+      }
+    } else {
+      for (int j = tid; j < n; j += CT) {
+        const uint32_t x = pb[j];
+        if ((x & mask) == prefix) atomicAdd(&sh.hist[w][(x >> shift) & 255u], 1u);
+      }
     }
     __syncthreads();
-    {
+    for (int b = tid; b < 256; b += CT) {
       uint32_t t = 0;
 #pragma unroll
-      for (int ww = 0; ww < 8; ++ww) t += sh.hist[ww][tid];
-      sh.tot[tid] = t;
+      for (int ww = 0; ww < (CT / 32); ++ww) t += sh.hist[ww][b];
+      sh.tot[b] = t;
     }
     __syncthreads();
     if (w == 0) {  // lanes walk bins from the top, 8 each
@@ -292,26 +313,27 @@ __device__ void select_rank(const uint32_t* pb, int n, int k, SelShared& sh, uin
 // CDF cut: the score v* of the lowest-ranked kept block and the fixed-point
 // mass strictly below v* ("below"), or found = false when the whole row's
 // mass stays under thr.
-__device__ void select_mass(const uint32_t* pb, int n, uint64_t thr, SelShared& sh, uint32_t& v,
+template <int CT>
+__device__ void select_mass(const uint32_t* pb, int n, uint64_t thr, SelShared<CT>& sh, uint32_t& v,
                             uint64_t& below, bool& found) {
   const int tid = threadIdx.x, w = tid / 32, lane = tid % 32;
   uint32_t prefix = 0, mask = 0;
   uint64_t blw = 0;
   found = true;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 8 * 256; b += kCT) (&sh.hsum[0][0])[b] = 0ull;
+    for (int b = tid; b < (CT / 32) * 256; b += CT) (&sh.hsum[0][0])[b] = 0ull;
     __syncthreads();
-    for (int j = tid; j < n; j += kCT) {
+    for (int j = tid; j < n; j += CT) {
       const uint32_t x = pb[j];
       if ((x & mask) == prefix)
         atomicAdd(&sh.hsum[w][(x >> shift) & 255u], static_cast<unsigned long long>(to_fixed(x)));
     }
     __syncthreads();
-    {
+    for (int b = tid; b < 256; b += CT) {
       unsigned long long t = 0;
 #pragma unroll
-      for (int ww = 0; ww < 8; ++ww) t += sh.hsum[ww][tid];
-      sh.tots[tid] = t;
+      for (int ww = 0; ww < (CT / 32); ++ww) t += sh.hsum[ww][b];
+      sh.tots[b] = t;
     }
     __syncthreads();
     if (w == 0) {  // lanes walk bins from the bottom, 8 each
@@ -355,9 +377,10 @@ __device__ void select_mass(const uint32_t* pb, int n, uint64_t thr, SelShared& 
 }
 
 // Largest pattern strictly below v (0 if none).
+template <int CT>
 __device__ uint32_t max_below(const uint32_t* pb, int n, uint32_t v, uint32_t* redu) {
   uint32_t m = 0;
-  for (int j = threadIdx.x; j < n; j += kCT) {
+  for (int j = threadIdx.x; j < n; j += CT) {
     const uint32_t x = pb[j];
     if (x < v && x > m) m = x;
   }
@@ -367,18 +390,19 @@ __device__ uint32_t max_below(const uint32_t* pb, int n, uint32_t v, uint32_t* r
   if (threadIdx.x % 32 == 0) redu[threadIdx.x / 32] = m;
   __syncthreads();
   uint32_t r = 0;
-  for (int i = 0; i < kCT / 32; ++i) r = max(r, redu[i]);
+  for (int i = 0; i < CT / 32; ++i) r = max(r, redu[i]);
   return r;
 }
 
 // Label pass: in index order, a block is in the top `take` ranks when its
 // pattern exceeds v, or equals v and fewer than `fill` lower-indexed blocks
 // also equal v.  `lab` gets `val` for those (and keeps larger labels).
+template <int CT>
 __device__ void label_top(const uint32_t* pb, int n, uint32_t v, int fill, int8_t* lab,
                           int8_t val, int* wsum) {
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
   int base = 0;
-  for (int j0 = 0; j0 < n; j0 += kCT) {
+  for (int j0 = 0; j0 < n; j0 += CT) {
     const int j = j0 + threadIdx.x;
     const uint32_t x = j < n ? pb[j] : 0u;
     const bool eq = j < n && x == v;
@@ -387,7 +411,7 @@ __device__ void label_top(const uint32_t* pb, int n, uint32_t v, int fill, int8_
     if (l == 0) wsum[w] = __popc(be);
     __syncthreads();
     int off = base, tot = 0;
-    for (int i = 0; i < kCT / 32; ++i) {
+    for (int i = 0; i < CT / 32; ++i) {
       if (i < w) off += wsum[i];
       tot += wsum[i];
     }
@@ -398,13 +422,14 @@ __device__ void label_top(const uint32_t* pb, int n, uint32_t v, int fill, int8_
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__ logits,
+template <int CT>
+__global__ void __launch_bounds__(CT) classify_kernel(const float* __restrict__ logits,
                                                        ClassifyArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int nkb = a.nkb, tid = threadIdx.x;
   uint32_t* pb = reinterpret_cast<uint32_t*>(smem);
   int8_t* lab = reinterpret_cast<int8_t*>(pb + nkb);
-  __shared__ SelShared sh;
+  __shared__ SelShared<CT> sh;
   __shared__ float redf[32];
   __shared__ int redi[32];
   __shared__ uint32_t redu[32];
@@ -415,14 +440,14 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
   float m = 0.f, inv = 1.f;
   if (!a.from_prob) {
     m = -FLT_MAX;
-    for (int j = tid; j < nkb; j += kCT) m = fmaxf(m, lr[j]);
-    m = block_reduce_max(m, redf);
+    for (int j = tid; j < nkb; j += CT) m = fmaxf(m, lr[j]);
+    m = block_reduce_max<CT>(m, redf);
     float se = 0.f;
-    for (int j = tid; j < nkb; j += kCT) se += expf(lr[j] - m);
-    se = block_reduce_sum(se, redf);
+    for (int j = tid; j < nkb; j += CT) se += expf(lr[j] - m);
+    se = block_reduce_sum<CT>(se, redf);
     inv = 1.0f / se;
   }
-  for (int j = tid; j < nkb; j += kCT) {
+  for (int j = tid; j < nkb; j += CT) {
     const float p = a.from_prob ? fmaxf(lr[j], 0.f) : expf(lr[j] - m) * inv;
     if (a.scores) a.scores[i64(row) * nkb + j] = p;
     pb[j] = __float_as_uint(p);
@@ -438,14 +463,14 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
     if (c > 0) {
       uint32_t v;
       int above;
-      select_rank(pb, nkb, c - 1, sh, v, above);
-      label_top(pb, nkb, v, c - above, lab, 2, redi);
+      select_rank<CT>(pb, nkb, c - 1, sh, v, above);
+      label_top<CT>(pb, nkb, v, c - above, lab, 2, redi);
       if (a.tie_count && c < nkb) {  // gap between ranks c-1 and c
-        const uint32_t nxt = max_below(pb, nkb, v, redu);
+        const uint32_t nxt = max_below<CT>(pb, nkb, v, redu);
         // rank c shares v when v's group is not exhausted by the cut
         int eqcount = 0;
-        for (int j = tid; j < nkb; j += kCT) eqcount += pb[j] == v;
-        eqcount = block_reduce_sum_int(eqcount, redi);
+        for (int j = tid; j < nkb; j += CT) eqcount += pb[j] == v;
+        eqcount = block_reduce_sum_int<CT>(eqcount, redi);
         const float hi = __uint_as_float(v);
         const float lo = (above + eqcount > c) ? hi : __uint_as_float(nxt);
         tie |= (hi - lo) <= kTieEps * hi;
@@ -455,9 +480,9 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
     uint32_t v = 0;
     uint64_t below = 0;
     bool found = false;
-    if (a.thr_fx > 0) select_mass(pb, nkb, a.thr_fx, sh, v, below, found);
+    if (a.thr_fx > 0) select_mass<CT>(pb, nkb, a.thr_fx, sh, v, below, found);
     if (a.thr_fx == 0) {
-      for (int j = tid; j < nkb; j += kCT) lab[j] = 2;  // nothing can be dropped
+      for (int j = tid; j < nkb; j += CT) lab[j] = 2;  // nothing can be dropped
       c = nkb;
       __syncthreads();
     } else {
@@ -468,8 +493,8 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
         // the r lowest-ranked (highest-index) ones are still below thr when
         // taken alone, the other g - r + 1 are kept
         int g = 0;
-        for (int j = tid; j < nkb; j += kCT) g += pb[j] == v;
-        g = block_reduce_sum_int(g, redi);
+        for (int j = tid; j < nkb; j += CT) g += pb[j] == v;
+        g = block_reduce_sum_int<CT>(g, redi);
         const uint64_t fx = to_fixed(v);
         const uint64_t r = (a.thr_fx - below + fx - 1) / fx;
         vk = v;
@@ -477,22 +502,22 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
       } else {
         // the row's whole mass stays below thr: only the top rank is kept
         uint32_t mx = 0;
-        for (int j = tid; j < nkb; j += kCT) mx = max(mx, pb[j]);
+        for (int j = tid; j < nkb; j += CT) mx = max(mx, pb[j]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         __syncthreads();
         if (tid % 32 == 0) redu[tid / 32] = mx;
         __syncthreads();
         mx = 0;
-        for (int i = 0; i < kCT / 32; ++i) mx = max(mx, redu[i]);
+        for (int i = 0; i < CT / 32; ++i) mx = max(mx, redu[i]);
         vk = mx;
         fill = 1;
       }
-      label_top(pb, nkb, vk, fill, lab, 2, redi);
+      label_top<CT>(pb, nkb, vk, fill, lab, 2, redi);
       int above = 0, eqc = 0;
-      for (int j = tid; j < nkb; j += kCT) { above += pb[j] > vk; eqc += pb[j] == vk; }
-      above = block_reduce_sum_int(above, redi);
-      eqc = block_reduce_sum_int(eqc, redi);
+      for (int j = tid; j < nkb; j += CT) { above += pb[j] > vk; eqc += pb[j] == vk; }
+      above = block_reduce_sum_int<CT>(above, redi);
+      eqc = block_reduce_sum_int<CT>(eqc, redi);
       c = above + fill;
       if (a.tie_count && found) {
         const double thr = static_cast<double>(a.thr_fx) / kFixedOne;
@@ -504,7 +529,7 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
         if (c < nkb) {
           tie |= fabs(thr - t_next) <= kTieEps;
           const float hi = __uint_as_float(vk);
-          const float lo = r >= 2 ? hi : __uint_as_float(max_below(pb, nkb, vk, redu));
+          const float lo = r >= 2 ? hi : __uint_as_float(max_below<CT>(pb, nkb, vk, redu));
           tie |= (hi - lo) <= kTieEps * hi;
         }
       }
@@ -515,13 +540,13 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
   if (nm > 0) {
     uint32_t v;
     int above;
-    select_rank(pb, nkb, c + nm - 1, sh, v, above);
-    label_top(pb, nkb, v, c + nm - above, lab, 1, redi);
+    select_rank<CT>(pb, nkb, c + nm - 1, sh, v, above);
+    label_top<CT>(pb, nkb, v, c + nm - above, lab, 1, redi);
     if (a.tie_count && c + nm < nkb) {
-      const uint32_t nxt = max_below(pb, nkb, v, redu);
+      const uint32_t nxt = max_below<CT>(pb, nkb, v, redu);
       int eqcount = 0;
-      for (int j = tid; j < nkb; j += kCT) eqcount += pb[j] == v;
-      eqcount = block_reduce_sum_int(eqcount, redi);
+      for (int j = tid; j < nkb; j += CT) eqcount += pb[j] == v;
+      eqcount = block_reduce_sum_int<CT>(eqcount, redi);
       const float hi = __uint_as_float(v);
       const float lo = (above + eqcount > c + nm) ? hi : __uint_as_float(nxt);
       tie |= (hi - lo) <= kTieEps * hi;
@@ -531,9 +556,9 @@ __global__ void __launch_bounds__(kCT) classify_kernel(const float* __restrict__
   __syncthreads();
 
   // 3. mask row and lists
-  for (int j = tid; j < nkb; j += kCT) a.mask[i64(row) * nkb + j] = lab[j];
+  for (int j = tid; j < nkb; j += CT) a.mask[i64(row) * nkb + j] = lab[j];
   const i64 off = i64(row) * nkb;
-  compact_row(lab, nkb, a.rows.crit_idx + off, a.rows.crit_cnt + row,
+  compact_row<CT>(lab, nkb, a.rows.crit_idx + off, a.rows.crit_cnt + row,
               a.rows.marg_idx + off, a.rows.marg_cnt + row, redi);
 }
 
@@ -552,15 +577,24 @@ cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
   a.scores = scores;
   a.tie_count = tie_count;
   const size_t smem = static_cast<size_t>(g.nkb) * 5 + 16;
-  cudaError_t e = cudaFuncSetAttribute(classify_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   if (tie_count) {
     e = cudaMemsetAsync(tie_count, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
   }
-  classify_kernel<<<g.BH * g.nqb, kCT, smem, s>>>(logits, a);
+  // short rows: small CTAs (cheap barriers, many rows per SM); long rows:
+  // more threads per row
+  if (g.nkb <= 1024) {
+    if ((e = cudaFuncSetAttribute(classify_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(smem))) != cudaSuccess)
+      return e;
+    classify_kernel<64><<<g.BH * g.nqb, 64, smem, s>>>(logits, a);
+  } else {
+    if ((e = cudaFuncSetAttribute(classify_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(smem))) != cudaSuccess)
+      return e;
+    classify_kernel<256><<<g.BH * g.nqb, 256, smem, s>>>(logits, a);
+  }
   return cudaGetLastError();
 }
 
@@ -577,7 +611,7 @@ __global__ void __launch_bounds__(kCT) rows_from_mask_kernel(const int8_t* __res
   for (int j = threadIdx.x; j < nkb; j += kCT) lab[j] = mask[i64(row) * nkb + j];
   __syncthreads();
   const i64 off = i64(row) * nkb;
-  compact_row(lab, nkb, rows.crit_idx + off, rows.crit_cnt + row,
+  compact_row<kCT>(lab, nkb, rows.crit_idx + off, rows.crit_cnt + row,
               rows.marg_idx + off, rows.marg_cnt + row, wsum);
 }
 
