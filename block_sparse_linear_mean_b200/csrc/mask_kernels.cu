@@ -66,50 +66,58 @@ cudaError_t launch_pool(const void* x, int dtype, float* out, int BH, int N,
 
 // ---------------------------------------------------------------------------
 // Pooled logits: logits[bh, i, j] = scale * <qbar[bh, i], kbar[bh, j]>, a
-// small fp32 GEMM (64 x 64 tile per CTA, 4 x 4 per thread, sequential
+// small fp32 GEMM (64 x 64 tile per CTA, 8 x 8 per thread, sequential
 // accumulation over d so every entry has a fixed summation order).
 
-__global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ qbar,
-                                                     const float* __restrict__ kbar,
-                                                     float* __restrict__ logits,
-                                                     int nqb, int nkb, int d,
-                                                     float scale) {
-  __shared__ float As[16][64 + 4];
-  __shared__ float Bs[16][64 + 4];
+__global__ void __launch_bounds__(64) logits_kernel(const float* __restrict__ qbar,
+                                                    const float* __restrict__ kbar,
+                                                    float* __restrict__ logits,
+                                                    int nqb, int nkb, int d,
+                                                    float scale) {
+  // 64 threads per 64 x 64 tile, 8 x 8 entries per thread; pooled rows are
+  // staged transposed ([k][row]) 32 channels at a time
+  __shared__ __align__(16) float As[32][64 + 4];
+  __shared__ __align__(16) float Bs[32][64 + 4];
   const int bh = blockIdx.z, i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
   const float* A = qbar + i64(bh) * nqb * d;
   const float* Bm = kbar + i64(bh) * nkb * d;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int kk = 0; kk < d; kk += 16) {
-    for (int e = threadIdx.x; e < 64 * 16; e += 256) {
-      const int r = e / 16, c = e % 16;
+  const int tid = threadIdx.x, tx = tid % 8, ty = tid / 8;
+  float acc[8][8] = {};
+  for (int kk = 0; kk < d; kk += 32) {
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {  // 64 rows x 8 float4 per operand
+      const int e = it * 64 + tid, r = e / 8, c4 = e % 8;
       const int gi = i0 + r, gj = j0 + r;
-      As[c][r] = gi < nqb ? A[i64(gi) * d + kk + c] : 0.f;
-      Bs[c][r] = gj < nkb ? Bm[i64(gj) * d + kk + c] : 0.f;
+      const float4 va = gi < nqb ? *reinterpret_cast<const float4*>(A + i64(gi) * d + kk + 4 * c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 vb = gj < nkb ? *reinterpret_cast<const float4*>(Bm + i64(gj) * d + kk + 4 * c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      As[4 * c4][r] = va.x; As[4 * c4 + 1][r] = va.y; As[4 * c4 + 2][r] = va.z; As[4 * c4 + 3][r] = va.w;
+      Bs[4 * c4][r] = vb.x; Bs[4 * c4 + 1][r] = vb.y; Bs[4 * c4 + 2][r] = vb.z; Bs[4 * c4 + 3][r] = vb.w;
     }
     __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {  // channels in order: a fixed summation order per entry
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[c][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[c][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8 + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      float a[4], b[4];
+      for (int m = 0; m < 8; ++m)
 #pragma unroll
-      for (int m = 0; m < 4; ++m) a[m] = As[c][ty * 4 + m];
-#pragma unroll
-      for (int n = 0; n < 4; ++n) b[n] = Bs[c][tx * 4 + n];
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int n = 0; n < 4; ++n) acc[m][n] = fmaf(a[m], b[n], acc[m][n]);
+        for (int n = 0; n < 8; ++n) acc[m][n] = fmaf(a[m], b[n], acc[m][n]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int gi = i0 + ty * 4 + m;
+  for (int m = 0; m < 8; ++m) {
+    const int gi = i0 + ty * 8 + m;
     if (gi >= nqb) continue;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      const int gj = j0 + tx * 4 + n;
+    for (int n = 0; n < 8; ++n) {
+      const int gj = j0 + tx * 8 + n;
       if (gj < nkb) logits[(i64(bh) * nqb + gi) * nkb + gj] = scale * acc[m][n];
     }
   }
@@ -118,8 +126,7 @@ __global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ q
 cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
                           const Geom& g, cudaStream_t s) {
   dim3 grid((g.nkb + 63) / 64, (g.nqb + 63) / 64, g.BH);
-  logits_kernel<<<grid, 256, 0, s>>>(qbar, kbar, logits, g.nqb, g.nkb, g.d,
-                                     g.scale);
+  logits_kernel<<<grid, 64, 0, s>>>(qbar, kbar, logits, g.nqb, g.nkb, g.d, g.scale);
   return cudaGetLastError();
 }
 
