@@ -30,6 +30,7 @@
 // status word gets SLA_ERR_TIMEOUT and all roles leave.
 #include <math.h>
 
+#include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -98,23 +99,47 @@ __device__ __forceinline__ void teardown(const BwdShared& sh, int warp, uint32_t
 }
 
 // ------------------------------------------------------------------ dQ
+// Query side of the linear branch, fused into the dq kernel's epilogue
+// (d = 128): for the tile's query block(s) i with marginal set M_i,
+//   g = dO W^T, den = phi(q) . z^M_i, dnum = g / den, dden = -(g . o) / den,
+//   dq += (dnum H^M_i^T + dden z^M_i) o phi'(q),
+//   dH^M_i = phi(Q_i)^T dnum,  dz^M_i = sum_t phi(q_t) dden_t.
+// marg_cnt == nullptr: no linear branch.
+struct LinBwdQ {
+  const float* zm;          // [B*H*Nqb, 128] z^M
+  const int32_t* marg_cnt;  // [B*H*Nqb]
+  const float* o_lin;       // [B*H, N, 128] saved O_lin
+  const __nv_bfloat16* q;   // [B*H, N, 128] (for phi')
+  __nv_bfloat16* dhm;       // [B*H*Nqb, 128, 128] out
+  float* dzm;               // [B*H*Nqb, 128] out
+  int nqb;
+};
+
 template <int D, int BQ, int BK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmHM, const __grid_constant__ CUtensorMap tmW,
                       const int32_t* __restrict__ tile_cnt, const uint32_t* __restrict__ tiles,
                       int plan_stride, const float* __restrict__ lse,
-                      const float* __restrict__ delta, float* __restrict__ dq, int32_t* status,
-                      int N, int nqt, float scale, float scale_log2, long long timeout) {
+                      const float* __restrict__ delta, float* __restrict__ dq, LinBwdQ lq,
+                      int32_t* status, int N, int nqt, float scale, float scale_log2,
+                      long long timeout) {
   constexpr int DC = D / 64;
   constexpr uint32_t kTileBytes = DC * 16384;  // 128 rows x D bf16 (Q, dO)
   constexpr uint32_t kHalfBytes = DC * 8192;   // 64 rows x D bf16 (K, V)
   constexpr uint32_t kStageBytes = 2 * kHalfBytes;
   constexpr uint32_t offQ = 0, offdO = kTileBytes, offKV = 2 * kTileBytes;
   constexpr uint32_t offBar = offKV + kBwdStages * kStageBytes;
-  constexpr uint32_t kUsed = offBar + 256;
+  constexpr uint32_t offRed = offBar + 512;   // [4][128] fp32 exchange slots
+  constexpr uint32_t offDd = offRed + 2048;   // [128] dden per row
+  constexpr uint32_t kUsed = offDd + 512;
   constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
   constexpr uint32_t idesc_dq = idesc_bf16(128, D, 0, 1);
+  // linear epilogue: after the main loop the K/V stages hold W (0), H^M of
+  // the tile's first and second query block (1, 2) and the bf16 dnum (3)
+  constexpr uint32_t offW = offKV, offHA = offKV + kStageBytes, offHB = offKV + 2 * kStageBytes;
+  constexpr uint32_t offDn = offKV + 3 * kStageBytes;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -130,7 +155,21 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   const uint32_t b_done = smem_u32(&bars[5 + 2 * kBwdStages]);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[6 + 2 * kBwdStages]);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[7 + 2 * kBwdStages]);
-  static_assert((8 + 2 * kBwdStages) * 8 <= 256, "barrier block");
+  // linear epilogue (single use each)
+  constexpr int kL0 = 8 + 2 * kBwdStages;
+  const uint32_t b_lin = smem_u32(&bars[kL0]);       // W, H^M landed
+  const uint32_t b_g = smem_u32(&bars[kL0 + 1]);     // g in TMEM
+  const uint32_t b_den = smem_u32(&bars[kL0 + 2]);   // den halves exchanged (8 warps)
+  const uint32_t b_go = smem_u32(&bars[kL0 + 3]);    // g . o halves exchanged (8 warps)
+  const uint32_t b_dn = smem_u32(&bars[kL0 + 4]);    // dnum and phi(Q) in smem (8 warps)
+  const uint32_t b_df = smem_u32(&bars[kL0 + 5]);    // df in TMEM
+  const uint32_t b_dh1 = smem_u32(&bars[kL0 + 6]);   // dH^M of the first block in TMEM
+  const uint32_t b_dfr = smem_u32(&bars[kL0 + 7]);   // df read (8 warps)
+  const uint32_t b_dh2 = smem_u32(&bars[kL0 + 8]);   // dH^M of the second block in TMEM
+  const uint32_t b_dz = smem_u32(&bars[kL0 + 9]);    // dz^M halves exchanged (8 warps)
+  static_assert((kL0 + 10) * 8 <= 512, "barrier block");
+  float* red = reinterpret_cast<float*>(base + offRed);
+  float* dd = reinterpret_cast<float*>(base + offDd);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int tile = blockIdx.x;
@@ -143,6 +182,17 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const uint32_t desc = ptiles[t];
     U += 1 + (step_of<BK>(desc, 1, N).present ? 1 : 0);
   }
+  // linear branch of the tile's query blocks (A: rows 0-63 or the whole
+  // 128-row block; B: rows 64-127 when blocks are 64 rows)
+  const bool lin_on = D == 128 && lq.marg_cnt != nullptr;
+  const int qa = BQ == 128 ? qt : 2 * qt;
+  const int qb2 = (BQ == 64 && 2 * qt + 1 < lq.nqb) ? 2 * qt + 1 : -1;
+  int nm_a = 0, nm_b = 0;
+  if (lin_on) {
+    nm_a = lq.marg_cnt[bh * lq.nqb + qa];
+    if (qb2 >= 0) nm_b = lq.marg_cnt[bh * lq.nqb + qb2];
+  }
+  const bool lin = nm_a > 0 || nm_b > 0;
 
   if (pad + kUsed > kBwdSmemRequest) {
     if (threadIdx.x == 0) atomicExch(status, static_cast<int32_t>(SLA_ERR_UNSUPPORTED));
@@ -159,6 +209,16 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       mbar_init(b_ds(b), 8);
     }
     mbar_init(b_done, 1);
+    mbar_init(b_lin, 1);
+    mbar_init(b_g, 1);
+    mbar_init(b_den, 8);
+    mbar_init(b_go, 8);
+    mbar_init(b_dn, 8);
+    mbar_init(b_df, 1);
+    mbar_init(b_dh1, 1);
+    mbar_init(b_dfr, 8);
+    mbar_init(b_dh2, 1);
+    mbar_init(b_dz, 8);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -176,7 +236,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   BwdShared sh{bars, abort_flag, status, timeout};
 
   if (warp == 0) {
-    if (lane == 0 && U > 0) {
+    if (lane == 0 && (U > 0 || lin)) {
       mbar_expect_tx(b_q, 2 * kTileBytes);
 #pragma unroll
       for (int c = 0; c < DC; ++c) {
@@ -200,6 +260,25 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             tma_load_3d(dst + kHalfBytes + c * 8192, &tmV, c * 64, st.row0, bh, b_full(s));
           }
           ++u;
+        }
+      }
+      // linear epilogue: W and H^M into the K/V stages once every dQ MMA
+      // (the stages' last readers) has completed
+      if constexpr (D == 128) {
+        if (ok && lin && (U == 0 || bwait(sh, b_done, 0))) {
+          mbar_expect_tx(b_lin, 32768u + (nm_a > 0 ? 32768u : 0u) + (nm_b > 0 ? 32768u : 0u));
+          tma_load_2d(sb + offW, &tmW, 0, 0, b_lin);
+          tma_load_2d(sb + offW + 16384, &tmW, 64, 0, b_lin);
+          if (nm_a > 0) {
+            const int hr = (bh * lq.nqb + qa) * 128;
+            tma_load_2d(sb + offHA, &tmHM, 0, hr, b_lin);
+            tma_load_2d(sb + offHA + 16384, &tmHM, 64, hr, b_lin);
+          }
+          if (nm_b > 0) {
+            const int hr = (bh * lq.nqb + qb2) * 128;
+            tma_load_2d(sb + offHB, &tmHM, 0, hr, b_lin);
+            tma_load_2d(sb + offHB + 16384, &tmHM, 64, hr, b_lin);
+          }
         }
       }
     }
@@ -247,6 +326,64 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         if (ok) ok = issue_dq(u);
       }
       if (ok) tc_commit(b_done);
+    }
+    if constexpr (D == 128) {
+      if (lane == 0 && lin) {
+        // g = dO W^T -> columns 384.. (M = 128 rows, N = 128, K = 128)
+        bool ok = bwait(sh, b_lin, 0) && bwait(sh, b_q, 0);
+        constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t id_mn = idesc_bf16(128, 128, 1, 1);
+        const uint64_t ddO = sdesc(sb + offdO, 16, 1024), dW = sdesc(sb + offW, 16, 1024);
+        const uint64_t dDn = sdesc(sb + offDn, 16, 1024), dDnmn = sdesc(sb + offDn, 16384, 1024);
+        const uint64_t dHA = sdesc(sb + offHA, 16, 1024), dHB = sdesc(sb + offHB, 16, 1024);
+        const uint64_t dPhimn = sdesc(sb + offQ, 16384, 1024);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t o = (kk / 4) * 16384 + (kk % 4) * 32;
+            tc_mma(tmem + 384, sdesc_add(ddO, o), sdesc_add(dW, o), id_kk, kk > 0);
+          }
+          tc_commit(b_g);
+          ok = bwait(sh, b_dn, 0);
+        }
+        if (ok) {
+          // df = dnum H^M^T (M = rows, N = channels a, K = c): block A into
+          // columns 0.., block B into 128..
+          tc_fence_after();
+          for (int q2 = 0; q2 < 2; ++q2) {
+            if ((q2 == 0 ? nm_a : nm_b) <= 0) continue;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t o = (kk / 4) * 16384 + (kk % 4) * 32;
+              tc_mma(tmem + 128u * q2, sdesc_add(dDn, o), sdesc_add(q2 == 0 ? dHA : dHB, o), id_kk,
+                     kk > 0);
+            }
+          }
+          tc_commit(b_df);
+          // dH^M of block A = phi(Q_A)^T dnum_A (M = a, N = c, K = its rows),
+          // into columns 384.. (g has been read)
+          constexpr int kRowsA = BQ == 128 ? 128 : 64;
+          if (nm_a > 0) {
+#pragma unroll
+            for (int kk = 0; kk < kRowsA / 16; ++kk)
+              tc_mma(tmem + 384, sdesc_add(dPhimn, kk * 2048), sdesc_add(dDnmn, kk * 2048), id_mn,
+                     kk > 0);
+          }
+          tc_commit(b_dh1);
+          if (BQ == 64 && nm_b > 0) {  // block B's rows 64-127, into columns 0.. once df is read
+            ok = bwait(sh, b_dfr, 0);
+            if (ok) {
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                tc_mma(tmem, sdesc_add(dPhimn, 8192 + kk * 2048), sdesc_add(dDnmn, 8192 + kk * 2048),
+                       id_mn, kk > 0);
+              tc_commit(b_dh2);
+            }
+          }
+        }
+      }
     }
   } else {
     const int h = (warp - 2) >> 2;  // key half of each step
@@ -315,8 +452,134 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     if (fin && U > 0) tc_fence_after();
     constexpr int DH = D / 2;
     const i64 orow = (static_cast<i64>(bh) * N + row) * D + h * DH;
+    bool lin_done = false;  // dq written by the linear epilogue
+    if constexpr (D == 128) {
+      if (lin && fin) {
+        // this thread: row r, channels [64h, 64h + 64)
+        const bool second = BQ == 64 && r >= 64;
+        const int nm_r = second ? nm_b : nm_a;
+        float4 z4[16];
+        if (nm_r > 0) {
+          const float4* zp = reinterpret_cast<const float4*>(
+              lq.zm + (static_cast<i64>(bh) * lq.nqb + (second ? qb2 : qa)) * 128 + h * 64);
 #pragma unroll
-    for (int c = 0; c < DH; c += 32) {
+          for (int i = 0; i < 16; ++i) z4[i] = __ldg(zp + i);
+        }
+        bool lok = __all_sync(full, bwait(sh, b_q, 0));
+        // phi(Q) in place, and this half of den = phi(q) . z^M from the same
+        // rounded values (as the forward forms it)
+        float dpart = 0.f, dpart2 = 0.f;
+        if (lok) {
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8) {
+            uint4* pq = reinterpret_cast<uint4*>(base + offQ + h * 16384 + sw128(r, u8));
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (row < N && nm_r > 0) {
+              val = phi_unit(*pq);
+              const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.x));
+              const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.y));
+              const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.z));
+              const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.w));
+              const float4 za = z4[2 * u8], zb = z4[2 * u8 + 1];
+              dpart = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, fmaf(f1.y, za.w, dpart))));
+              dpart2 = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, dpart2))));
+            }
+            *pq = val;
+          }
+          red[h * 128 + r] = dpart + dpart2;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_den);
+          lok = __all_sync(full, bwait(sh, b_den, 0));
+        }
+        const float den = lok ? dpart + dpart2 + red[(h ^ 1) * 128 + r] : 0.f;
+        const float dinv = (nm_r > 0 && den > 0.f && row < N) ? 1.f / den : 0.f;
+        // g and this half of g . o
+        if (lok) lok = __all_sync(full, bwait(sh, b_g, 0));
+        float gv[64];
+        float go = 0.f;
+        if (lok) {
+          tc_fence_after();
+          tmem_ld32(tmem + 384 + lane_off + h * 64, gv);
+          tmem_ld32(tmem + 384 + lane_off + h * 64 + 32, gv + 32);
+          tmem_wait_ld();
+          reg_fence<64>(gv);
+          if (row < N && nm_r > 0) {
+            const float4* op = reinterpret_cast<const float4*>(
+                lq.o_lin + (static_cast<i64>(bh) * N + row) * 128 + h * 64);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float4 o4 = __ldg(op + i);
+              go = fmaf(gv[4 * i], o4.x, fmaf(gv[4 * i + 1], o4.y,
+                        fmaf(gv[4 * i + 2], o4.z, fmaf(gv[4 * i + 3], o4.w, go))));
+            }
+          }
+          red[(2 + h) * 128 + r] = go;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_go);
+          lok = __all_sync(full, bwait(sh, b_go, 0));
+        }
+        const float ddn = lok ? -(go + red[(2 + (h ^ 1)) * 128 + r]) * dinv : 0.f;
+        if (lok) {
+          // dnum = g / den (bf16) into the K-major [row][c] tile
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8)
+            *reinterpret_cast<uint4*>(base + offDn + h * 16384 + sw128(r, u8)) = make_uint4(
+                pack_bf16x2(gv[8 * u8] * dinv, gv[8 * u8 + 1] * dinv),
+                pack_bf16x2(gv[8 * u8 + 2] * dinv, gv[8 * u8 + 3] * dinv),
+                pack_bf16x2(gv[8 * u8 + 4] * dinv, gv[8 * u8 + 5] * dinv),
+                pack_bf16x2(gv[8 * u8 + 6] * dinv, gv[8 * u8 + 7] * dinv));
+          if (h == 0) dd[r] = ddn;
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_dn);
+          lok = __all_sync(full, bwait(sh, b_df, 0));
+        }
+        if (lok) {
+          // dq = s dQ + (df + dden z^M) o phi'(q), written once
+          tc_fence_after();
+          const uint32_t tdf = tmem + (second ? 128u : 0u);
+          const __nv_bfloat16* qrow = lq.q + (static_cast<i64>(bh) * N + row) * 128 + h * 64;
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            float dfv[32], dqv[32];
+            if (nm_r > 0) tmem_ld32(tdf + lane_off + h * 64 + c0, dfv);
+            if (U > 0) tmem_ld32(tQ + lane_off + h * 64 + c0, dqv);
+            tmem_wait_ld();
+            reg_fence<32>(dfv);
+            reg_fence<32>(dqv);
+            if (row < N) {
+#pragma unroll
+              for (int i8 = 0; i8 < 4; ++i8) {
+                const uint4 qu = *reinterpret_cast<const uint4*>(qrow + c0 + 8 * i8);
+                const uint32_t qw[4] = {qu.x, qu.y, qu.z, qu.w};
+                float ov[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[e]));
+                  const int c = c0 + 8 * i8 + 2 * e;
+                  const float zx = reinterpret_cast<const float*>(&z4[c / 4])[c % 4];
+                  const float zy = reinterpret_cast<const float*>(&z4[c / 4])[c % 4 + 1];
+                  const float base0 = U > 0 ? scale * dqv[8 * i8 + 2 * e] : 0.f;
+                  const float base1 = U > 0 ? scale * dqv[8 * i8 + 2 * e + 1] : 0.f;
+                  ov[2 * e] = nm_r > 0 ? base0 + (dfv[8 * i8 + 2 * e] + ddn * zx) * dphi(qf.x) : base0;
+                  ov[2 * e + 1] = nm_r > 0 ? base1 + (dfv[8 * i8 + 2 * e + 1] + ddn * zy) * dphi(qf.y) : base1;
+                }
+                float* dst = dq + orow + c0 + 8 * i8;
+                *reinterpret_cast<float4*>(dst) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(ov[4], ov[5], ov[6], ov[7]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_dfr);
+          lin_done = true;
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; !lin_done && c < DH; c += 32) {
       float o[32];
       if (fin && U > 0) {
         tmem_ld32(tQ + lane_off + h * DH + c, o);
@@ -332,6 +595,66 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
           *reinterpret_cast<float4*>(dq + orow + c + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+      }
+    }
+    if constexpr (D == 128) {
+      if (lin_on && fin) {
+        // dH^M (bf16) and dz^M of the tile's query blocks; zeros for blocks
+        // without marginal sets (the key side's gather reads every block).
+        // Accumulator lane = channel a.  64-row blocks: half h writes block h;
+        // a 128-row block: half h writes columns [64h, 64h + 64) and sums
+        // dz^M over rows [64h, 64h + 64).
+        const int a = quad * 32 + lane;
+        const int bsel = BQ == 64 ? h : 0;
+        const int qblk = bsel == 0 ? qa : qb2;
+        const int nmb = bsel == 0 ? nm_a : nm_b;
+        const bool have = nmb > 0 && lin_done;
+        if (qblk >= 0) {
+          __nv_bfloat16* dst = lq.dhm + (static_cast<i64>(bh) * lq.nqb + qblk) * 16384 + a * 128;
+          constexpr int kCN = BQ == 64 ? 128 : 64;
+          const int clo = BQ == 64 ? 0 : h * 64;
+          bool hok = have;
+          if (have) hok = __all_sync(full, bwait(sh, bsel == 0 ? b_dh1 : b_dh2, 0));
+          if (hok) tc_fence_after();
+          const uint32_t tsrc = (bsel == 0 ? tmem + 384 : tmem) + lane_off;
+#pragma unroll
+          for (int c0 = 0; c0 < kCN; c0 += 32) {
+            float v[32];
+            if (hok) {
+              tmem_ld32(tsrc + clo + c0, v);
+              tmem_wait_ld();
+              reg_fence<32>(v);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              *reinterpret_cast<uint4*>(dst + clo + c0 + 8 * q4) =
+                  make_uint4(pack_bf16x2(v[8 * q4], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                             pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+          }
+          // dz^M[a] = sum over the block's rows of phi(Q)[row][a] dden[row]
+          float dz = 0.f;
+          if (hok) {
+            const int r0 = BQ == 64 ? 64 * bsel : 64 * h;
+            const uint8_t* chunk = base + offQ + (a >> 6) * 16384;
+            for (int rr = r0; rr < r0 + 64; ++rr) {
+              const uint16_t bits =
+                  *reinterpret_cast<const uint16_t*>(chunk + sw128(rr, (a & 63) >> 3) + (a & 7) * 2);
+              dz = fmaf(__uint_as_float(static_cast<uint32_t>(bits) << 16), dd[rr], dz);
+            }
+          }
+          float* zdst = lq.dzm + (static_cast<i64>(bh) * lq.nqb + qblk) * 128 + a;
+          if (BQ == 64) {
+            *zdst = dz;
+          } else {
+            red[h * 128 + a] = dz;  // (slot 0-1: den was read before the dnum barrier)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_dz);
+            if (__all_sync(full, bwait(sh, b_dz, 0)) && h == 0) *zdst = dz + red[128 + a];
+          }
+        }
       }
     }
   }
@@ -634,7 +957,8 @@ BwdPlans bwd_plans(const Geom& g, void* scratch) {
 }
 
 template <int D, int BQ, int BK>
-cudaError_t launch_bwd_t(const CUtensorMap* m128, const CUtensorMap* m64, const BwdPlans& pl,
+cudaError_t launch_bwd_t(const CUtensorMap* m128, const CUtensorMap* m64, const CUtensorMap& mhm,
+                         const CUtensorMap& mw, const LinBwdQ& lq, const BwdPlans& pl,
                          const float* lse, const float* delta, float* dq, float* dk, float* dv,
                          int32_t* status, const Geom& g, cudaStream_t s) {
   const int nt = (g.N + 127) / 128;
@@ -646,9 +970,9 @@ cudaError_t launch_bwd_t(const CUtensorMap* m128, const CUtensorMap* m64, const 
   cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kBwdSmemRequest));
   if (e != cudaSuccess) return e;
-  kq<<<g.BH * nt, kBwdThreads, kBwdSmemRequest, s>>>(m128[0], m128[3], m64[1], m64[2], pl.qcnt,
-                                                     pl.qtiles, g.nkb, lse, delta, dq, status, g.N,
-                                                     nt, g.scale, scale_log2, timeout);
+  kq<<<g.BH * nt, kBwdThreads, kBwdSmemRequest, s>>>(m128[0], m128[3], m64[1], m64[2], mhm, mw,
+                                                     pl.qcnt, pl.qtiles, g.nkb, lse, delta, dq, lq,
+                                                     status, g.N, nt, g.scale, scale_log2, timeout);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   auto kk = attn_bwd_dkdv_tc_kernel<D, BQ, BK>;
@@ -669,8 +993,9 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
                                const float* lse, const float* delta,
                                const sla_block_lists& rows, const sla_block_lists& cols,
                                float* dq, float* dk, float* dv, const Geom& g, void* scratch,
-                               int32_t* status, cudaStream_t s) {
+                               int32_t* status, cudaStream_t s, const LinBwdIn* lin) {
   if (!attn_tc_supported(g)) return cudaErrorNotSupported;
+  if (lin && g.d != 128) return cudaErrorNotSupported;
   const BwdPlans pl = bwd_plans(g, scratch);
   cudaError_t e = launch_tile_plan(rows, g.BH, g.nqb, g.nkb, g.bq, g.bk, pl.qcnt, pl.qtiles, s);
   if (e != cudaSuccess) return e;
@@ -681,9 +1006,26 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   for (int i = 0; i < 4; ++i)
     if (!make_rows_map(&m128[i], src[i], g, 128) || !make_rows_map(&m64[i], src[i], g, 64))
       return cudaErrorInvalidValue;
+  // the linear branch's query side runs in the dq kernel's epilogue
+  CUtensorMap mhm = m128[0], mw = m128[0];  // placeholders when it is off
+  LinBwdQ lq{};
+  lq.nqb = g.nqb;
+  if (lin) {
+    const uint64_t dhm[2] = {128, static_cast<uint64_t>(g.BH) * g.nqb * 128}, dw2[2] = {128, 128};
+    const uint64_t s2[1] = {256};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_bf16_map(&mhm, lin->hm, 2, dhm, s2, box) || !encode_bf16_map(&mw, lin->wb, 2, dw2, s2, box))
+      return cudaErrorInvalidValue;
+    lq.zm = lin->zm;
+    lq.marg_cnt = lin->marg_cnt;
+    lq.o_lin = lin->o_lin;
+    lq.q = static_cast<const __nv_bfloat16*>(q);
+    lq.dhm = static_cast<__nv_bfloat16*>(lin->dhm);
+    lq.dzm = lin->dzm;
+  }
 #define SLA_BWD_CASE(D_, BQ_, BK_)                  \
   if (g.d == D_ && g.bq == BQ_ && g.bk == BK_)      \
-    return launch_bwd_t<D_, BQ_, BK_>(m128, m64, pl, lse, delta, dq, dk, dv, status, g, s);
+    return launch_bwd_t<D_, BQ_, BK_>(m128, m64, mhm, mw, lq, pl, lse, delta, dq, dk, dv, status, g, s);
   SLA_BWD_CASE(128, 64, 64)
   SLA_BWD_CASE(128, 64, 128)
   SLA_BWD_CASE(128, 128, 64)

@@ -69,14 +69,27 @@ constexpr uint32_t kPlanPresent = 1u << 15;
 cudaError_t launch_tile_plan(const sla_block_lists& lists, int BH, int nrb, int ncb, int rb,
                              int cb, int32_t* cnt, uint32_t* tiles, cudaStream_t s);
 
+// Linear-branch inputs of the fused query side of the backward (d = 128).
+struct LinBwdIn {
+  const void* hm;           // [B*H*Nqb, 128, 128] bf16 H^M (forward prepare)
+  const void* wb;           // [128, 128] bf16 W
+  const float* zm;          // [B*H*Nqb, 128] z^M
+  const int32_t* marg_cnt;  // [B*H*Nqb] marginal counts
+  const float* o_lin;       // [B*H, N, 128] saved O_lin
+  void* dhm;                // out: [B*H*Nqb, 128, 128] bf16 dH^M
+  float* dzm;               // out: [B*H*Nqb, 128] dz^M
+};
+
 // backward of the critical branch on the tensor cores (attn_bwd_tc.cu):
-// dq, dk, dv are overwritten (fp32); the linear branch adds to them later.
+// dq, dk, dv are overwritten (fp32).  With `lin`, the dq kernel also adds
+// the linear branch's dq and writes dH^M, dz^M for the key side; dk, dv get
+// the linear branch later (launch_lin_bwd_kv).
 size_t attn_bwd_tc_scratch_bytes(const Geom& g);
 cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
                                const float* lse, const float* delta,
                                const sla_block_lists& rows, const sla_block_lists& cols,
                                float* dq, float* dk, float* dv, const Geom& g, void* scratch,
-                               int32_t* status, cudaStream_t s);
+                               int32_t* status, cudaStream_t s, const LinBwdIn* lin);
 // Outputs of the fused tensor-core attention; any pointer may be null.
 struct AttnOutputs {
   float* o_s;     // fp32 O_s
@@ -130,10 +143,16 @@ cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, i
 size_t lin_bwd_tc_scratch_bytes(const Geom& g);
 cudaError_t launch_delta(const void* dout, const float* o_s, float* delta, const Geom& g,
                          cudaStream_t s);
-cudaError_t launch_lin_bwd_tc(const void* q, const void* k, const void* v, const float* proj,
-                              const void* dout, const sla_block_lists& rows,
-                              const sla_block_lists& cols, const float* o_lin, float* dq,
-                              float* dk, float* dv, float* dproj, const Geom& g, void* scratch,
+// 1. before the attention backward: H^M, z^M, W in bf16 into `scratch`, and
+//    the pointers the fused query side needs
+cudaError_t launch_lin_bwd_prepare(const void* k, const void* v, const float* proj,
+                                   const sla_block_lists& rows, const float* o_lin,
+                                   const Geom& g, void* scratch, int32_t* status,
+                                   cudaStream_t s, LinBwdIn* lin);
+// 2. after it: the key side (dH gather, dk, dv) and dW
+cudaError_t launch_lin_bwd_kv(const void* k, const void* v, const void* dout,
+                              const sla_block_lists& cols, const float* o_lin, float* dk,
+                              float* dv, float* dproj, const Geom& g, void* scratch,
                               int32_t* status, cudaStream_t s);
 
 // backward

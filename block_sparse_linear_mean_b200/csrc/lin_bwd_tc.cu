@@ -19,14 +19,15 @@
 // in the forward, so the backward differentiates the forward's own
 // arithmetic; g, dnum, dH^M and dH go through bf16 once as MMA operands.
 //
-// Kernels (all waits bounded; timeouts set the status word):
-//   delta_kernel        Delta_t = dO_t . O_s[t]                (HBM-bound)
-//   dw_tc_kernel        dW partials, persistent over 128-token tiles
-//   lin_bwd_q_tc_kernel one CTA per query block with marginal blocks
-//   lin_bwd_kv_tc_kernel one CTA per key block that is marginal somewhere
-// The two block kernels work transposed (TMEM lane = channel, column =
-// token), so per-token scalars are column factors and per-channel sums are
-// thread-local.
+// Kernels here (all waits bounded; timeouts set the status word):
+//   delta_kernel         Delta_t = dO_t . O_s[t]                (HBM-bound)
+//   dw_tc_kernel         dW partials, persistent over 128-token tiles
+//   lin_bwd_kv_tc_kernel one CTA per key block that is marginal somewhere,
+//                        working transposed (TMEM lane = channel, column =
+//                        token)
+// The query side (g, dnum, dq, dH^M, dz^M) runs in the epilogue of the
+// critical branch's dq kernel (attn_bwd_tc.cu), where Q, dO and dQ already
+// sit on chip.
 #include <algorithm>
 
 #include "common.cuh"
@@ -44,36 +45,6 @@ constexpr int kLHElems = kLD * kLD;  // one d x d matrix
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
   const uint32_t a = smem_u32(p);
   return p + (((a + 1023u) & ~1023u) - a);
-}
-
-// element `col` (0..127) of row `row` in a tile stored as two 128B-swizzled
-// chunks of 64 columns, `chunk` bytes apart
-__device__ __forceinline__ uint32_t sw_off(int row, int col, uint32_t chunk) {
-  return (col >> 6) * chunk + sw128(row, (col & 63) >> 3) + (col & 7) * 2;
-}
-__device__ __forceinline__ float bf16_load(const uint8_t* tile, int row, int col, uint32_t chunk) {
-  const uint16_t bits = *reinterpret_cast<const uint16_t*>(tile + sw_off(row, col, chunk));
-  return __uint_as_float(static_cast<uint32_t>(bits) << 16);
-}
-__device__ __forceinline__ void bf16_store(uint8_t* tile, int row, int col, uint32_t chunk, float x) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(x);
-  *reinterpret_cast<__nv_bfloat16*>(tile + sw_off(row, col, chunk)) = b;
-}
-
-// Butterfly reduce-scatter over the warp: on entry each lane holds v[0..31];
-// on exit v[0] of lane L is the warp's sum of v[L].
-__device__ __forceinline__ void warp_reduce_scatter32(float* v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const float send = up ? v[i] : v[i + off];
-      const float keep = up ? v[i + off] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -212,202 +183,6 @@ __global__ void dw_sum_kernel(const float* __restrict__ part, float* __restrict_
   float s = 0.f;
   for (int p = 0; p < nparts; ++p) s += part[static_cast<i64>(p) * kLHElems + i];
   dproj[i] = s;
-}
-
-// ---------------------------------------------------------------------------
-// Query side: one CTA (128 threads, thread = channel) per (query block i, bh)
-// with marginal blocks.
-//   1. g^T   = W dO^T            (M = 128 channels c, N = BQ tokens, K = 128)
-//   2. den_t from the rounded phi(q_t) (as the forward), (g . o)_t by a
-//      reduce-scatter over channels, dden_t = -(g . o)_t / den_t,
-//      dnum = g / den -> bf16 [t][c] tile (in W's place)
-//   3. df^T  = H^M dnum^T        (M = 128 channels a, N = BQ, K = 128 c)
-//      dH^M  = phi(Q)^T dnum     (M = 128 a, N = 128 c, K = BQ tokens)
-//   4. dq_t += (df_t + dden_t z^M) o phi'(q_t);  dH^M (bf16) and
-//      dz^M_i = sum_t phi(q_t) dden_t (fp32) to global for the key side.
-template <int BQ>
-__global__ void __launch_bounds__(128) lin_bwd_q_tc_kernel(
-    const __grid_constant__ CUtensorMap tmHM, const __grid_constant__ CUtensorMap tmW,
-    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
-    const float* __restrict__ zmar, const int32_t* __restrict__ marg_cnt,
-    const __nv_bfloat16* __restrict__ q, const float* __restrict__ o_lin, float* __restrict__ dq,
-    __nv_bfloat16* __restrict__ dhm, float* __restrict__ dzm, int N, int nqb, int nkb,
-    int32_t* status) {
-  constexpr uint32_t kQC = BQ * 128;                 // one 64-channel chunk of a BQ-row tile
-  constexpr uint32_t offHM = 0, offW = 32768;        // W, later dnum [t][c]
-  constexpr uint32_t offQ = 65536, offdO = offQ + 2 * kQC;
-  constexpr uint32_t offSc = offdO + 2 * kQC;        // per-token scalars, z^M
-  constexpr uint32_t offBar = offSc + 4096;
-  constexpr uint32_t kCols = 256;                     // g^T / df^T at 0, dH^M at BQ
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = align1k(smem_raw);
-  const uint32_t sb = smem_u32(base);
-  float* den = reinterpret_cast<float*>(base + offSc);   // [BQ]
-  float* part = den + BQ;                                // [4][BQ]
-  float* dden = part + 4 * BQ;                           // [BQ]
-  float* zm = dden + BQ;                                 // [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
-  const uint32_t b_tma = smem_u32(&bars[0]), b_m1 = smem_u32(&bars[1]), b_m2 = smem_u32(&bars[2]);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(&bars[3]);
-  const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int list_row = bh * nqb + i;
-  if (min(max(marg_cnt[list_row], 0), nkb) == 0) {
-    // no marginal blocks: nothing to add to dq; dH^M_i, dz^M_i are zero (the
-    // gather multiplies every row, with indicator 0 for this one, and must
-    // not meet uninitialised memory)
-    uint4* dst = reinterpret_cast<uint4*>(dhm + static_cast<i64>(list_row) * kLHElems);
-    for (int x = tid; x < kLHElems / 8; x += 128) dst[x] = make_uint4(0u, 0u, 0u, 0u);
-    dzm[static_cast<i64>(list_row) * kLD + tid] = 0.f;
-    return;
-  }
-  const int t0g = i * BQ, valid = min(BQ, N - t0g);
-  if (tid == 0) {
-    mbar_init(b_tma, 1);
-    mbar_init(b_m1, 1);
-    mbar_init(b_m2, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) tmem_alloc(smem_u32(tslot), kCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const int c = tid;
-  bool ok = true;
-  if (tid == 0) {
-    mbar_expect_tx(b_tma, 2 * 32768 + 4 * kQC);
-    const int hrow = list_row * kLD;
-    tma_load_2d(sb + offHM, &tmHM, 0, hrow, b_tma);
-    tma_load_2d(sb + offHM + 16384, &tmHM, 64, hrow, b_tma);
-    tma_load_2d(sb + offW, &tmW, 0, 0, b_tma);
-    tma_load_2d(sb + offW + 16384, &tmW, 64, 0, b_tma);
-    tma_load_3d(sb + offQ, &tmQ, 0, t0g, bh, b_tma);
-    tma_load_3d(sb + offQ + kQC, &tmQ, 64, t0g, bh, b_tma);
-    tma_load_3d(sb + offdO, &tmdO, 0, t0g, bh, b_tma);
-    tma_load_3d(sb + offdO + kQC, &tmdO, 64, t0g, bh, b_tma);
-  }
-  zm[c] = zmar[static_cast<i64>(list_row) * kLD + c];
-  ok = __syncthreads_and(wait_bounded(b_tma, 0, status, kLbTimeout));
-  if (ok && tid == 0) {  // 1. g^T = W dO^T
-    tc_fence_after();
-    constexpr uint32_t idesc = idesc_bf16(128, BQ, 0, 0);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      tc_mma(tmem, sdesc(sb + offW + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-             sdesc(sb + offdO + (kk >> 2) * kQC + (kk & 3) * 32, 16, 1024), idesc, kk > 0);
-    tc_commit(b_m1);
-  }
-  if (ok) {
-    // phi(Q) in place (rows past N zero), then the normalisers from it
-    for (int x = tid; x < BQ * 16; x += 128) {
-      const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
-      uint4* p = reinterpret_cast<uint4*>(base + offQ + chunk * kQC + sw128(row, u));
-      *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    __syncthreads();
-    for (int t = tid; t < BQ; t += 128) {
-      float s = 0.f;
-      for (int a = 0; a < kLD; ++a) s += bf16_load(base + offQ, t, a, kQC) * zm[a];
-      den[t] = s;
-    }
-    ok = __syncthreads_and(wait_bounded(b_m1, 0, status, kLbTimeout));
-  }
-  if (ok) {
-    // 2. g (lane c, column t) -> (g . o)_t partials per warp, dnum tile
-    tc_fence_after();
-    uint8_t* dn = base + offW;  // W is consumed: b_m1 completed
-#pragma unroll
-    for (int tt = 0; tt < BQ; tt += 32) {
-      float gv[32], pr[32];
-      tmem_ld32(tmem + lane_off + tt, gv);
-      tmem_wait_ld();
-      reg_fence<32>(gv);
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int t = tt + k;
-        const bool in = t < valid;
-        const float o = in ? o_lin[(static_cast<i64>(bh) * N + t0g + t) * kLD + c] : 0.f;
-        pr[k] = gv[k] * o;
-        const float dv = den[t];
-        bf16_store(dn, t, c, kQC, (in && dv > 0.f) ? gv[k] / dv : 0.f);
-      }
-      warp_reduce_scatter32(pr);
-      part[warp * BQ + tt + lane] = pr[0];
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    for (int t = tid; t < BQ; t += 128) {
-      const float go = (part[t] + part[BQ + t]) + (part[2 * BQ + t] + part[3 * BQ + t]);
-      dden[t] = (t < valid && den[t] > 0.f) ? -go / den[t] : 0.f;
-    }
-    if (tid == 0) {  // 3. df^T = H^M dnum^T and dH^M = phi(Q)^T dnum
-      tc_fence_after();
-      constexpr uint32_t idf = idesc_bf16(128, BQ, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma(tmem, sdesc(sb + offHM + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-               sdesc(sb + offW + (kk >> 2) * kQC + (kk & 3) * 32, 16, 1024), idf, kk > 0);
-      constexpr uint32_t idh = idesc_bf16(128, 128, 1, 1);
-#pragma unroll
-      for (int kk = 0; kk < BQ / 16; ++kk)
-        tc_mma(tmem + BQ, sdesc(sb + offQ + kk * 2048, kQC, 1024), sdesc(sb + offW + kk * 2048, kQC, 1024),
-               idh, kk > 0);
-      tc_commit(b_m2);
-    }
-    __syncthreads();  // dden visible to every thread
-    // dz^M_i[a] = sum_t phi(q_t)[a] dden_t   (thread a = c)
-    float dz = 0.f;
-    for (int t = 0; t < valid; ++t) dz += bf16_load(base + offQ, t, c, kQC) * dden[t];
-    dzm[static_cast<i64>(list_row) * kLD + c] = dz;
-    ok = __syncthreads_and(wait_bounded(b_m2, 0, status, kLbTimeout));
-  }
-  if (ok) {
-    // 4. dq += (df + dden z^M) o phi'(q)   (lane a, column t)
-    tc_fence_after();
-    const float za = zm[c];
-#pragma unroll
-    for (int tt = 0; tt < BQ; tt += 32) {
-      float dfv[32];
-      tmem_ld32(tmem + lane_off + tt, dfv);
-      tmem_wait_ld();
-      reg_fence<32>(dfv);
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int t = tt + k;
-        if (t < valid) {
-          const i64 off = (static_cast<i64>(bh) * N + t0g + t) * kLD + c;
-          const float x = __bfloat162float(q[off]);
-          dq[off] += (dfv[k] + dden[t] * za) * dphi(x);
-        }
-      }
-    }
-    // dH^M row a -> global bf16
-    __nv_bfloat16* dst = dhm + static_cast<i64>(list_row) * kLHElems + c * kLD;
-#pragma unroll
-    for (int c0 = 0; c0 < kLD; c0 += 32) {
-      float v[32];
-      tmem_ld32(tmem + BQ + lane_off + c0, v);
-      tmem_wait_ld();
-      reg_fence<32>(v);
-#pragma unroll
-      for (int k = 0; k < 32; k += 8)
-        *reinterpret_cast<uint4*>(dst + c0 + k) =
-            make_uint4(pack_bf16x2(v[k], v[k + 1]), pack_bf16x2(v[k + 2], v[k + 3]),
-                       pack_bf16x2(v[k + 4], v[k + 5]), pack_bf16x2(v[k + 6], v[k + 7]));
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (!ok) {
-    const long long t0 = clock64();
-    while (clock64() - t0 < 2000000) __nanosleep(1000);
-  }
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kCols);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -564,54 +339,52 @@ cudaError_t launch_delta(const void* dout, const float* o_s, float* delta, const
   return cudaGetLastError();
 }
 
-cudaError_t launch_lin_bwd_tc(const void* q, const void* k, const void* v, const float* proj,
-                              const void* dout, const sla_block_lists& rows,
-                              const sla_block_lists& cols, const float* o_lin, float* dq,
-                              float* dk, float* dv, float* dproj, const Geom& g, void* scratch,
+cudaError_t launch_lin_bwd_prepare(const void* k, const void* v, const float* proj,
+                                   const sla_block_lists& rows, const float* o_lin,
+                                   const Geom& g, void* scratch, int32_t* status,
+                                   cudaStream_t s, LinBwdIn* lin) {
+  if (!lin_tc_supported(g)) return cudaErrorNotSupported;
+  const LinBwdWs w = lin_bwd_ws(g);
+  char* sc = static_cast<char*>(scratch);
+  cudaError_t e = launch_lin_tc_prepare(k, v, proj, rows, g, sc + w.lin, status, s);
+  if (e != cudaSuccess) return e;
+  const LinInputs li = lin_tc_inputs(g, sc + w.lin, rows);
+  lin->hm = li.hm;
+  lin->wb = li.wb;
+  lin->zm = li.zm;
+  lin->marg_cnt = rows.marg_cnt;
+  lin->o_lin = o_lin;
+  lin->dhm = sc + w.dhm;
+  lin->dzm = reinterpret_cast<float*>(sc + w.dzm);
+  return cudaSuccess;
+}
+
+cudaError_t launch_lin_bwd_kv(const void* k, const void* v, const void* dout,
+                              const sla_block_lists& cols, const float* o_lin, float* dk,
+                              float* dv, float* dproj, const Geom& g, void* scratch,
                               int32_t* status, cudaStream_t s) {
   if (!lin_tc_supported(g)) return cudaErrorNotSupported;
   const LinBwdWs w = lin_bwd_ws(g);
   char* sc = static_cast<char*>(scratch);
-  const uint64_t BH = g.BH, N = g.N, nqb = g.nqb, nkb = g.nkb;
+  const uint64_t BH = g.BH, N = g.N, nkb = g.nkb;
   cudaError_t e;
   if (g.linear) {
-    if ((e = launch_lin_tc_prepare(k, v, proj, rows, g, sc + w.lin, status, s)) != cudaSuccess)
-      return e;
-    const LinInputs li = lin_tc_inputs(g, sc + w.lin, rows);
-    CUtensorMap mHM, mW, mQ, mdO, mDH, mK, mV;
-    const uint64_t dq3[3] = {kLD, N, BH}, sq3[2] = {kLD * 2, N * kLD * 2};
-    const uint32_t boxq[3] = {64, static_cast<uint32_t>(g.bq), 1};
-    const uint32_t boxk[3] = {64, static_cast<uint32_t>(g.bk), 1};
-    const uint64_t dhm[2] = {kLD, BH * nqb * kLD}, ddh[2] = {kLD, BH * nkb * kLD}, s2[1] = {kLD * 2};
-    const uint64_t dw2[2] = {kLD, kLD};
-    const uint32_t box2[2] = {64, 128};
-    if (!encode_bf16_map(&mHM, li.hm, 2, dhm, s2, box2) || !encode_bf16_map(&mW, li.wb, 2, dw2, s2, box2) ||
-        !encode_bf16_map(&mQ, q, 3, dq3, sq3, boxq) || !encode_bf16_map(&mdO, dout, 3, dq3, sq3, boxq) ||
-        !encode_bf16_map(&mDH, sc + w.dh, 2, ddh, s2, box2) ||
-        !encode_bf16_map(&mK, k, 3, dq3, sq3, boxk) || !encode_bf16_map(&mV, v, 3, dq3, sq3, boxk))
-      return cudaErrorInvalidValue;
-    __nv_bfloat16* dhm_p = reinterpret_cast<__nv_bfloat16*>(sc + w.dhm);
-    float* dzm_p = reinterpret_cast<float*>(sc + w.dzm);
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
-    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
-    dim3 gq(g.nqb, g.BH);
-    if (g.bq == 64) {
-      const size_t smem = 65536 + 4 * 64 * 128 + 4096 + 64 + 1024;
-      if ((e = lb_set_smem(lin_bwd_q_tc_kernel<64>, smem)) != cudaSuccess) return e;
-      lin_bwd_q_tc_kernel<64><<<gq, 128, smem, s>>>(mHM, mW, mQ, mdO, li.zm, rows.marg_cnt, qb, o_lin, dq,
-                                                    dhm_p, dzm_p, g.N, g.nqb, g.nkb, status);
-    } else {
-      const size_t smem = 65536 + 4 * 128 * 128 + 4096 + 64 + 1024;
-      if ((e = lb_set_smem(lin_bwd_q_tc_kernel<128>, smem)) != cudaSuccess) return e;
-      lin_bwd_q_tc_kernel<128><<<gq, 128, smem, s>>>(mHM, mW, mQ, mdO, li.zm, rows.marg_cnt, qb, o_lin, dq,
-                                                     dhm_p, dzm_p, g.N, g.nqb, g.nkb, status);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // dH_j, dz_j: the indicator GEMM over the column lists
-    if ((e = launch_list_gather(cols, g.BH, g.nkb, g.nqb, dhm_p, dzm_p, sc + w.dh,
+    // dH_j, dz_j: the indicator GEMM over the column lists (dH^M, dz^M were
+    // written by the dq kernel, zeros for query blocks without marginal sets)
+    if ((e = launch_list_gather(cols, g.BH, g.nkb, g.nqb, sc + w.dhm,
+                                reinterpret_cast<const float*>(sc + w.dzm), sc + w.dh,
                                 reinterpret_cast<float*>(sc + w.dz), sc + w.indt, w.ldt, status, s)) !=
         cudaSuccess)
       return e;
+    CUtensorMap mDH, mK, mV;
+    const uint64_t dq3[3] = {kLD, N, BH}, sq3[2] = {kLD * 2, N * kLD * 2};
+    const uint32_t boxk[3] = {64, static_cast<uint32_t>(g.bk), 1};
+    const uint64_t ddh[2] = {kLD, BH * nkb * kLD}, s2[1] = {kLD * 2};
+    const uint32_t box2[2] = {64, 128};
+    if (!encode_bf16_map(&mDH, sc + w.dh, 2, ddh, s2, box2) ||
+        !encode_bf16_map(&mK, k, 3, dq3, sq3, boxk) || !encode_bf16_map(&mV, v, 3, dq3, sq3, boxk))
+      return cudaErrorInvalidValue;
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
     dim3 gk(g.nkb, g.BH);
     const float* dz_p = reinterpret_cast<const float*>(sc + w.dz);
     if (g.bk == 64) {

@@ -410,11 +410,19 @@ sla_status sla_backward(const sla_params* p, const void* q, const void* k,
   float* delta = at<float>(ws, w.delta);
   int32_t* status = static_cast<int32_t*>(ws);
   if (bwd_tc_linear(g)) {
+    // Delta; the linear branch's H^M, z^M (as in the forward); the critical
+    // backward with the linear branch's query side fused into its dq kernel;
+    // then the linear branch's key side and dW
     SLA_CUDA(sla::launch_delta(dout, o_s, delta, g, s));
+    sla::LinBwdIn lin{};
+    const bool linear = has_linear_branch(g);
+    if (linear)
+      SLA_CUDA(sla::launch_lin_bwd_prepare(k, v, proj, *rows, o_lin, g, at<char>(ws, w.lin), status,
+                                           s, &lin));
     SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
-                                     at<char>(ws, w.plans), status, s));
-    SLA_CUDA(sla::launch_lin_bwd_tc(q, k, v, proj, dout, *rows, *cols, o_lin, dq, dk, dv, dproj, g,
-                                    at<char>(ws, w.lin), status, s));
+                                     at<char>(ws, w.plans), status, s, linear ? &lin : nullptr));
+    SLA_CUDA(sla::launch_lin_bwd_kv(k, v, dout, *cols, o_lin, dk, dv, dproj, g, at<char>(ws, w.lin),
+                                    status, s));
     return SLA_OK;
   }
   float* gbuf = at<float>(ws, w.gbuf);
@@ -422,7 +430,7 @@ sla_status sla_backward(const sla_params* p, const void* q, const void* k,
   SLA_CUDA(sla::launch_bwd_prep(dout, o_s, o_lin, proj, delta, gbuf, dwp, g, s));
   if (bwd_tc_attention(g)) {
     SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
-                                     at<char>(ws, w.plans), static_cast<int32_t*>(ws), s));
+                                     at<char>(ws, w.plans), static_cast<int32_t*>(ws), s, nullptr));
   } else {
     SLA_CUDA(sla::launch_attn_bwd_dq(q, k, v, dout, lse, delta, *rows, dq, g, s));
     SLA_CUDA(sla::launch_attn_bwd_dkdv(q, k, v, dout, lse, delta, *cols, dk, dv, g, s));
