@@ -290,10 +290,10 @@ def run_ours(args, rank, world, local_rank):
         lin = wl.frac_marg > 0
         launches_per_step += 1  # column lists
         if fused and wl.d == 128:
-            # Delta | 2 tile plans, dq, dkdv | (W to bf16, summaries,
-            # indicator, gather, linear q side, indicator + gather of dH,
-            # linear kv side, dW partials, dW sum)
-            launches_per_step += 1 + 4 + (10 if lin else 0)
+            # Delta | 2 tile plans, dq (+ linear query side), dkdv (+ linear
+            # key side) | (W to bf16, summaries, indicator, gather of H^M,
+            # indicator + gather of dH, dW partials, dW sum)
+            launches_per_step += 1 + 4 + (8 if lin else 0)
         else:
             # Delta and g, dW partials | dq, dkdv (tcgen05: + 2 tile plans) |
             # (summaries, linear dq, linear dk dv) | dW reduction

@@ -115,6 +115,18 @@ struct LinBwdQ {
   int nqb;
 };
 
+// Key side of the linear branch, fused into the dkdv kernel's epilogue
+// (d = 128): for the tile's key block(s) j that are marginal somewhere, with
+// dH_j, dz_j the sums of dH^M_i, dz^M_i over the query blocks i that hold j,
+//   dv += phi(K_j) dH_j,  dk += (V_j dH_j^T + dz_j) o phi'(k).
+// marg_cnt == nullptr: no linear branch.
+struct LinBwdK {
+  const float* dz;          // [B*H*Nkb, 128] dz_j
+  const int32_t* marg_cnt;  // [B*H*Nkb] per key block: query blocks holding it
+  const __nv_bfloat16* k;   // [B*H, N, 128] (for phi and phi')
+  int nkb;
+};
+
 template <int D, int BQ, int BK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
@@ -666,11 +678,12 @@ template <int D, int BQ, int BK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                        const __grid_constant__ CUtensorMap tmDH,
                         const int32_t* __restrict__ tile_cnt, const uint32_t* __restrict__ tiles,
                         int plan_stride, const float* __restrict__ lse,
                         const float* __restrict__ delta, float* __restrict__ dk,
-                        float* __restrict__ dv, int32_t* status, int N, int nkt, float scale,
-                        float scale_log2, long long timeout) {
+                        float* __restrict__ dv, LinBwdK lk, int32_t* status, int N, int nkt,
+                        float scale, float scale_log2, long long timeout) {
   constexpr int DC = D / 64;
   constexpr uint32_t kTileBytes = DC * 16384;  // 128 rows x D bf16 (K, V)
   constexpr uint32_t kHalfBytes = DC * 8192;   // 64 rows x D bf16 (Q, dO)
@@ -681,6 +694,11 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   constexpr uint32_t kUsed = offBar + 256;
   constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
   constexpr uint32_t idesc_g = idesc_bf16(128, D, 0, 1);
+  // linear epilogue: after the main loop the stages hold dH of the tile's
+  // first and second key block (0, 1) and, for 64-row blocks, phi(K) with
+  // the other block's rows zeroed (2: first block, 3: second)
+  constexpr uint32_t offDHA = offSt, offDHB = offSt + kStageBytes;
+  constexpr uint32_t offPhA = offSt + 2 * kStageBytes, offPhB = offSt + 3 * kStageBytes;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -696,7 +714,11 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   const uint32_t b_done = smem_u32(&bars[5 + 2 * kBwdStages]);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[6 + 2 * kBwdStages]);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[7 + 2 * kBwdStages]);
-  static_assert((8 + 2 * kBwdStages) * 8 <= 256, "barrier block");
+  constexpr int kL0 = 8 + 2 * kBwdStages;
+  const uint32_t b_lin = smem_u32(&bars[kL0]);       // dH landed
+  const uint32_t b_phk = smem_u32(&bars[kL0 + 1]);   // phi(K) in smem (8 warps)
+  const uint32_t b_lkv = smem_u32(&bars[kL0 + 2]);   // linear dV, dphi in TMEM
+  static_assert((kL0 + 3) * 8 <= 256, "barrier block");
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int tile = blockIdx.x;
@@ -705,6 +727,16 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   const uint32_t* ptiles = tiles + static_cast<i64>(tile) * plan_stride;
   int U = 0;
   for (int t = 0; t < T; ++t) U += 1 + (step_of<BQ>(ptiles[t], 1, N).present ? 1 : 0);
+  // linear branch of the tile's key blocks (A: rows 0-63 or the whole
+  // 128-row block; B: rows 64-127 when blocks are 64 rows)
+  const int ja = BK == 128 ? kt : 2 * kt;
+  const int jb = (BK == 64 && 2 * kt + 1 < lk.nkb) ? 2 * kt + 1 : -1;
+  int nm_a = 0, nm_b = 0;
+  if (D == 128 && lk.marg_cnt != nullptr) {
+    nm_a = lk.marg_cnt[bh * lk.nkb + ja];
+    if (jb >= 0) nm_b = lk.marg_cnt[bh * lk.nkb + jb];
+  }
+  const bool lin = nm_a > 0 || nm_b > 0;
 
   if (pad + kUsed > kBwdSmemRequest) {
     if (threadIdx.x == 0) atomicExch(status, static_cast<int32_t>(SLA_ERR_UNSUPPORTED));
@@ -721,6 +753,9 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       mbar_init(b_pd(b), 8);
     }
     mbar_init(b_done, 1);
+    mbar_init(b_lin, 1);
+    mbar_init(b_phk, 8);
+    mbar_init(b_lkv, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -740,7 +775,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   if (warp == 0) {
     // K and V tiles stay resident; the steps stream Q, dO and the per-query
     // -LSE*log2(e), -Delta (q >= N: -inf and 0, so those columns vanish)
-    if (U > 0) {
+    if (U > 0 || lin) {
       if (lane == 0) {
         mbar_expect_tx(b_kv, 2 * kTileBytes);
 #pragma unroll
@@ -785,6 +820,23 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           __syncwarp();
           if (lane == 0) mbar_arrive(b_full(s));
           ++u;
+        }
+      }
+      // linear epilogue: dH of the tile's key blocks into stages 0 and 1
+      // once every MMA of the main loop (the stages' last readers) completed
+      if constexpr (D == 128) {
+        if (lane == 0 && ok && lin && (U == 0 || bwait(sh, b_done, 0))) {
+          mbar_expect_tx(b_lin, (nm_a > 0 ? 32768u : 0u) + (nm_b > 0 ? 32768u : 0u));
+          if (nm_a > 0) {
+            const int hr = (bh * lk.nkb + ja) * 128;
+            tma_load_2d(sb + offDHA, &tmDH, 0, hr, b_lin);
+            tma_load_2d(sb + offDHA + 16384, &tmDH, 64, hr, b_lin);
+          }
+          if (nm_b > 0) {
+            const int hr = (bh * lk.nkb + jb) * 128;
+            tma_load_2d(sb + offDHB, &tmDH, 0, hr, b_lin);
+            tma_load_2d(sb + offDHB + 16384, &tmDH, 64, hr, b_lin);
+          }
         }
       }
     }
@@ -836,6 +888,44 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         if (ok) ok = issue_grad(u);
       }
       if (ok) tc_commit(b_done);
+    }
+    if constexpr (D == 128) {
+      if (lane == 0 && lin) {
+        bool ok = bwait(sh, b_lin, 0) && bwait(sh, b_phk, 0);
+        if (ok) {
+          tc_fence_after();
+          constexpr uint32_t id_dv = idesc_bf16(128, 128, 0, 1);  // A phi(K) K-major, B dH MN-major
+          constexpr uint32_t id_dp = idesc_bf16(128, 128, 0, 0);  // A V, B dH rows: both K-major
+          const uint64_t dHAmn = sdesc(sb + offDHA, 16384, 1024), dHBmn = sdesc(sb + offDHB, 16384, 1024);
+          const uint64_t dHAk = sdesc(sb + offDHA, 16, 1024), dHBk = sdesc(sb + offDHB, 16, 1024);
+          const uint64_t dPhA = sdesc(sb + (BK == 128 ? offK : offPhA), 16, 1024);
+          const uint64_t dPhB = sdesc(sb + offPhB, 16, 1024);
+          const uint64_t dVd = sdesc(sb + offV, 16, 1024);
+          // dv += phi(K) dH (M = key rows, N = c, K = a), into the dV
+          // accumulator (written fresh when the tile had no critical step)
+          bool fresh = U == 0;
+          for (int q2 = 0; q2 < 2; ++q2) {
+            if ((q2 == 0 ? nm_a : nm_b) <= 0) continue;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma(tV, sdesc_add(q2 == 0 ? dPhA : dPhB, (kk / 4) * 16384 + (kk % 4) * 32),
+                     sdesc_add(q2 == 0 ? dHAmn : dHBmn, kk * 2048), id_dv, (fresh && kk == 0) ? 0u : 1u);
+            fresh = false;
+          }
+          // dphi = V dH^T (M = key rows, N = a, K = c): block A into
+          // columns 0.., block B into 128..
+          for (int q2 = 0; q2 < 2; ++q2) {
+            if ((q2 == 0 ? nm_a : nm_b) <= 0) continue;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t o = (kk / 4) * 16384 + (kk % 4) * 32;
+              tc_mma(tmem + 128u * q2, sdesc_add(dVd, o), sdesc_add(q2 == 0 ? dHAk : dHBk, o), id_dp,
+                     kk > 0);
+            }
+          }
+          tc_commit(b_lkv);
+        }
+      }
     }
   } else {
     const int h = (warp - 2) >> 2;  // query half of each step
@@ -895,8 +985,92 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     if (fin && U > 0) tc_fence_after();
     constexpr int DH = D / 2;
     const i64 orow = (static_cast<i64>(bh) * N + key) * D + h * DH;
+    bool lin_done = false;  // dk, dv written by the linear epilogue
+    if constexpr (D == 128) {
+      if (lin && fin) {
+        // this thread: key row r, channels [64h, 64h + 64)
+        const bool second = BK == 64 && r >= 64;
+        const int nm_r = second ? nm_b : nm_a;
+        const int jblk = second ? jb : ja;
+        bool lok = __all_sync(full, bwait(sh, b_kv, 0));
+        if (lok) {
+          // phi(K) (rows past N zero): in place for 128-row blocks; for
+          // 64-row blocks into the copy of the row's own block, zeros into
+          // the other's
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
+          for (int u8 = 0; u8 < 8; ++u8) {
+            uint4* pk = reinterpret_cast<uint4*>(base + offK + h * 16384 + sw128(r, u8));
+            const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+            const uint4 ph = key < N ? phi_unit(*pk) : zero;
+            if (BK == 128) {
+              *pk = ph;
+            } else {
+              *reinterpret_cast<uint4*>(base + offPhA + h * 16384 + sw128(r, u8)) = second ? zero : ph;
+              *reinterpret_cast<uint4*>(base + offPhB + h * 16384 + sw128(r, u8)) = second ? ph : zero;
+            }
+          }
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_phk);
+          lok = __all_sync(full, bwait(sh, b_lkv, 0));
+        }
+        if (lok) {
+          // dk = s dK + (dphi + dz) o phi'(k), dv = dV (the linear part is
+          // already in the accumulator)
+          tc_fence_after();
+          float4 z4[16];
+          if (nm_r > 0) {
+            const float4* zp = reinterpret_cast<const float4*>(
+                lk.dz + (static_cast<i64>(bh) * lk.nkb + jblk) * 128 + h * 64);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z4[i] = __ldg(zp + i);
+          }
+          const __nv_bfloat16* krow = lk.k + (static_cast<i64>(bh) * N + key) * 128 + h * 64;
+          const uint32_t tdp = tmem + (second ? 128u : 0u);
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            float kv[32], vv[32], dpv[32];
+            if (U > 0) tmem_ld32(tK + lane_off + h * 64 + c0, kv);
+            tmem_ld32(tV + lane_off + h * 64 + c0, vv);
+            if (nm_r > 0) tmem_ld32(tdp + lane_off + h * 64 + c0, dpv);
+            tmem_wait_ld();
+            reg_fence<32>(kv);
+            reg_fence<32>(vv);
+            reg_fence<32>(dpv);
+            if (key < N) {
+#pragma unroll
+              for (int i8 = 0; i8 < 4; ++i8) {
+                const uint4 ku = *reinterpret_cast<const uint4*>(krow + c0 + 8 * i8);
+                const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w};
+                float ok8[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw[e]));
+                  const int c = c0 + 8 * i8 + 2 * e;
+                  const float zx = reinterpret_cast<const float*>(&z4[c / 4])[c % 4];
+                  const float zy = reinterpret_cast<const float*>(&z4[c / 4])[c % 4 + 1];
+                  const float b0 = U > 0 ? scale * kv[8 * i8 + 2 * e] : 0.f;
+                  const float b1 = U > 0 ? scale * kv[8 * i8 + 2 * e + 1] : 0.f;
+                  ok8[2 * e] = nm_r > 0 ? b0 + (dpv[8 * i8 + 2 * e] + zx) * dphi(kf.x) : b0;
+                  ok8[2 * e + 1] = nm_r > 0 ? b1 + (dpv[8 * i8 + 2 * e + 1] + zy) * dphi(kf.y) : b1;
+                }
+                float* kd = dk + orow + c0 + 8 * i8;
+                *reinterpret_cast<float4*>(kd) = make_float4(ok8[0], ok8[1], ok8[2], ok8[3]);
+                *reinterpret_cast<float4*>(kd + 4) = make_float4(ok8[4], ok8[5], ok8[6], ok8[7]);
+                float* vd = dv + orow + c0 + 8 * i8;
+                *reinterpret_cast<float4*>(vd) = make_float4(vv[8 * i8], vv[8 * i8 + 1], vv[8 * i8 + 2], vv[8 * i8 + 3]);
+                *reinterpret_cast<float4*>(vd + 4) =
+                    make_float4(vv[8 * i8 + 4], vv[8 * i8 + 5], vv[8 * i8 + 6], vv[8 * i8 + 7]);
+              }
+            }
+          }
+          lin_done = true;
+        }
+      }
+    }
+#pragma unroll
+    for (int which = 0; !lin_done && which < 2; ++which) {
       float* dst = which == 0 ? dk : dv;
       const uint32_t src = which == 0 ? tK : tV;
       const float mul = which == 0 ? scale : 1.f;
@@ -957,10 +1131,10 @@ BwdPlans bwd_plans(const Geom& g, void* scratch) {
 }
 
 template <int D, int BQ, int BK>
-cudaError_t launch_bwd_t(const CUtensorMap* m128, const CUtensorMap* m64, const CUtensorMap& mhm,
-                         const CUtensorMap& mw, const LinBwdQ& lq, const BwdPlans& pl,
-                         const float* lse, const float* delta, float* dq, float* dk, float* dv,
-                         int32_t* status, const Geom& g, cudaStream_t s) {
+cudaError_t launch_dq_t(const CUtensorMap* m128, const CUtensorMap* m64, const CUtensorMap& mhm,
+                        const CUtensorMap& mw, const LinBwdQ& lq, const BwdPlans& pl,
+                        const float* lse, const float* delta, float* dq, int32_t* status,
+                        const Geom& g, cudaStream_t s) {
   const int nt = (g.N + 127) / 128;
   const float scale_log2 = g.scale * 1.4426950408889634f;
   const bool debug = (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0;
@@ -973,27 +1147,46 @@ cudaError_t launch_bwd_t(const CUtensorMap* m128, const CUtensorMap* m64, const 
   kq<<<g.BH * nt, kBwdThreads, kBwdSmemRequest, s>>>(m128[0], m128[3], m64[1], m64[2], mhm, mw,
                                                      pl.qcnt, pl.qtiles, g.nkb, lse, delta, dq, lq,
                                                      status, g.N, nt, g.scale, scale_log2, timeout);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int D, int BQ, int BK>
+cudaError_t launch_dkdv_t(const CUtensorMap* m128, const CUtensorMap* m64, const CUtensorMap& mdh,
+                          const LinBwdK& lk, const BwdPlans& pl, const float* lse,
+                          const float* delta, float* dk, float* dv, int32_t* status,
+                          const Geom& g, cudaStream_t s) {
+  const int nt = (g.N + 127) / 128;
+  const float scale_log2 = g.scale * 1.4426950408889634f;
+  const bool debug = (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0;
+  const long long timeout = debug ? (1ll << 24) : (1ll << 31);
   auto kk = attn_bwd_dkdv_tc_kernel<D, BQ, BK>;
-  e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kBwdSmemRequest));
+  cudaError_t e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kBwdSmemRequest));
   if (e != cudaSuccess) return e;
-  kk<<<g.BH * nt, kBwdThreads, kBwdSmemRequest, s>>>(m128[1], m128[2], m64[0], m64[3], pl.kcnt,
-                                                     pl.ktiles, g.nqb, lse, delta, dk, dv, status,
+  kk<<<g.BH * nt, kBwdThreads, kBwdSmemRequest, s>>>(m128[1], m128[2], m64[0], m64[3], mdh, pl.kcnt,
+                                                     pl.ktiles, g.nqb, lse, delta, dk, dv, lk, status,
                                                      g.N, nt, g.scale, scale_log2, timeout);
   return cudaGetLastError();
+}
+
+bool bwd_maps(const void* q, const void* k, const void* v, const void* dout, const Geom& g,
+              CUtensorMap* m128, CUtensorMap* m64) {
+  const void* src[4] = {q, k, v, dout};
+  for (int i = 0; i < 4; ++i)
+    if (!make_rows_map(&m128[i], src[i], g, 128) || !make_rows_map(&m64[i], src[i], g, 64))
+      return false;
+  return true;
 }
 
 }  // namespace
 
 size_t attn_bwd_tc_scratch_bytes(const Geom& g) { return bwd_plans(g, nullptr).bytes; }
 
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* lse, const float* delta,
-                               const sla_block_lists& rows, const sla_block_lists& cols,
-                               float* dq, float* dk, float* dv, const Geom& g, void* scratch,
-                               int32_t* status, cudaStream_t s, const LinBwdIn* lin) {
+cudaError_t launch_attn_bwd_tc_dq(const void* q, const void* k, const void* v, const void* dout,
+                                  const float* lse, const float* delta,
+                                  const sla_block_lists& rows, const sla_block_lists& cols,
+                                  float* dq, const Geom& g, void* scratch, int32_t* status,
+                                  cudaStream_t s, const LinBwdIn* lin) {
   if (!attn_tc_supported(g)) return cudaErrorNotSupported;
   if (lin && g.d != 128) return cudaErrorNotSupported;
   const BwdPlans pl = bwd_plans(g, scratch);
@@ -1002,10 +1195,7 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   e = launch_tile_plan(cols, g.BH, g.nkb, g.nqb, g.bk, g.bq, pl.kcnt, pl.ktiles, s);
   if (e != cudaSuccess) return e;
   CUtensorMap m128[4], m64[4];
-  const void* src[4] = {q, k, v, dout};
-  for (int i = 0; i < 4; ++i)
-    if (!make_rows_map(&m128[i], src[i], g, 128) || !make_rows_map(&m64[i], src[i], g, 64))
-      return cudaErrorInvalidValue;
+  if (!bwd_maps(q, k, v, dout, g, m128, m64)) return cudaErrorInvalidValue;
   // the linear branch's query side runs in the dq kernel's epilogue
   CUtensorMap mhm = m128[0], mw = m128[0];  // placeholders when it is off
   LinBwdQ lq{};
@@ -1023,18 +1213,52 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
     lq.dhm = static_cast<__nv_bfloat16*>(lin->dhm);
     lq.dzm = lin->dzm;
   }
-#define SLA_BWD_CASE(D_, BQ_, BK_)                  \
-  if (g.d == D_ && g.bq == BQ_ && g.bk == BK_)      \
-    return launch_bwd_t<D_, BQ_, BK_>(m128, m64, mhm, mw, lq, pl, lse, delta, dq, dk, dv, status, g, s);
-  SLA_BWD_CASE(128, 64, 64)
-  SLA_BWD_CASE(128, 64, 128)
-  SLA_BWD_CASE(128, 128, 64)
-  SLA_BWD_CASE(128, 128, 128)
-  SLA_BWD_CASE(64, 64, 64)
-  SLA_BWD_CASE(64, 64, 128)
-  SLA_BWD_CASE(64, 128, 64)
-  SLA_BWD_CASE(64, 128, 128)
-#undef SLA_BWD_CASE
+#define SLA_DQ_CALL(D_, BQ_, BK_) launch_dq_t<D_, BQ_, BK_>(m128, m64, mhm, mw, lq, pl, lse, delta, dq, status, g, s)
+#define SLA_DQ(...) SLA_DQ_CALL(__VA_ARGS__)
+  if (g.d == 128 && g.bq == 64 && g.bk == 64) return SLA_DQ(128, 64, 64);
+  if (g.d == 128 && g.bq == 64 && g.bk == 128) return SLA_DQ(128, 64, 128);
+  if (g.d == 128 && g.bq == 128 && g.bk == 64) return SLA_DQ(128, 128, 64);
+  if (g.d == 128 && g.bq == 128 && g.bk == 128) return SLA_DQ(128, 128, 128);
+  if (g.d == 64 && g.bq == 64 && g.bk == 64) return SLA_DQ(64, 64, 64);
+  if (g.d == 64 && g.bq == 64 && g.bk == 128) return SLA_DQ(64, 64, 128);
+  if (g.d == 64 && g.bq == 128 && g.bk == 64) return SLA_DQ(64, 128, 64);
+  if (g.d == 64 && g.bq == 128 && g.bk == 128) return SLA_DQ(64, 128, 128);
+#undef SLA_DQ
+#undef SLA_DQ_CALL
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_attn_bwd_tc_dkdv(const void* q, const void* k, const void* v,
+                                    const void* dout, const float* lse, const float* delta,
+                                    float* dk, float* dv, const Geom& g, void* scratch,
+                                    int32_t* status, cudaStream_t s, const LinBwdKIn* lin) {
+  if (!attn_tc_supported(g)) return cudaErrorNotSupported;
+  if (lin && g.d != 128) return cudaErrorNotSupported;
+  const BwdPlans pl = bwd_plans(g, scratch);  // built by launch_attn_bwd_tc_dq
+  CUtensorMap m128[4], m64[4];
+  if (!bwd_maps(q, k, v, dout, g, m128, m64)) return cudaErrorInvalidValue;
+  // the linear branch's key side runs in the dkdv kernel's epilogue
+  CUtensorMap mdh = m128[0];  // placeholder when it is off
+  LinBwdK lk{};
+  lk.nkb = g.nkb;
+  if (lin) {
+    const uint64_t ddh[2] = {128, static_cast<uint64_t>(g.BH) * g.nkb * 128}, s2[1] = {256};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_bf16_map(&mdh, lin->dh, 2, ddh, s2, box)) return cudaErrorInvalidValue;
+    lk.dz = lin->dz;
+    lk.marg_cnt = lin->marg_cnt;
+    lk.k = static_cast<const __nv_bfloat16*>(k);
+  }
+#define SLA_KV(D_, BQ_, BK_) launch_dkdv_t<D_, BQ_, BK_>(m128, m64, mdh, lk, pl, lse, delta, dk, dv, status, g, s)
+  if (g.d == 128 && g.bq == 64 && g.bk == 64) return SLA_KV(128, 64, 64);
+  if (g.d == 128 && g.bq == 64 && g.bk == 128) return SLA_KV(128, 64, 128);
+  if (g.d == 128 && g.bq == 128 && g.bk == 64) return SLA_KV(128, 128, 64);
+  if (g.d == 128 && g.bq == 128 && g.bk == 128) return SLA_KV(128, 128, 128);
+  if (g.d == 64 && g.bq == 64 && g.bk == 64) return SLA_KV(64, 64, 64);
+  if (g.d == 64 && g.bq == 64 && g.bk == 128) return SLA_KV(64, 64, 128);
+  if (g.d == 64 && g.bq == 128 && g.bk == 64) return SLA_KV(64, 128, 64);
+  if (g.d == 64 && g.bq == 128 && g.bk == 128) return SLA_KV(64, 128, 128);
+#undef SLA_KV
   return cudaErrorNotSupported;
 }
 

@@ -80,16 +80,28 @@ struct LinBwdIn {
   float* dzm;               // out: [B*H*Nqb, 128] dz^M
 };
 
-// backward of the critical branch on the tensor cores (attn_bwd_tc.cu):
-// dq, dk, dv are overwritten (fp32).  With `lin`, the dq kernel also adds
-// the linear branch's dq and writes dH^M, dz^M for the key side; dk, dv get
-// the linear branch later (launch_lin_bwd_kv).
+// Linear-branch inputs of the fused key side (d = 128).
+struct LinBwdKIn {
+  const void* dh;           // [B*H*Nkb, 128, 128] bf16 dH_j
+  const float* dz;          // [B*H*Nkb, 128] dz_j
+  const int32_t* marg_cnt;  // [B*H*Nkb] per key block: query blocks holding it
+};
+
+// backward of the critical branch on the tensor cores (attn_bwd_tc.cu), in
+// two launches.  _dq builds the row and column tile plans in `scratch` and
+// writes dq (fp32); with `lin` its epilogue adds the linear branch's dq and
+// writes dH^M, dz^M.  _dkdv (same scratch) writes dk, dv; with `lin` its
+// epilogue adds the linear branch's dk, dv.
 size_t attn_bwd_tc_scratch_bytes(const Geom& g);
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* lse, const float* delta,
-                               const sla_block_lists& rows, const sla_block_lists& cols,
-                               float* dq, float* dk, float* dv, const Geom& g, void* scratch,
-                               int32_t* status, cudaStream_t s, const LinBwdIn* lin);
+cudaError_t launch_attn_bwd_tc_dq(const void* q, const void* k, const void* v, const void* dout,
+                                  const float* lse, const float* delta,
+                                  const sla_block_lists& rows, const sla_block_lists& cols,
+                                  float* dq, const Geom& g, void* scratch, int32_t* status,
+                                  cudaStream_t s, const LinBwdIn* lin);
+cudaError_t launch_attn_bwd_tc_dkdv(const void* q, const void* k, const void* v,
+                                    const void* dout, const float* lse, const float* delta,
+                                    float* dk, float* dv, const Geom& g, void* scratch,
+                                    int32_t* status, cudaStream_t s, const LinBwdKIn* lin);
 // Outputs of the fused tensor-core attention; any pointer may be null.
 struct AttnOutputs {
   float* o_s;     // fp32 O_s
@@ -149,11 +161,14 @@ cudaError_t launch_lin_bwd_prepare(const void* k, const void* v, const float* pr
                                    const sla_block_lists& rows, const float* o_lin,
                                    const Geom& g, void* scratch, int32_t* status,
                                    cudaStream_t s, LinBwdIn* lin);
-// 2. after it: the key side (dH gather, dk, dv) and dW
-cudaError_t launch_lin_bwd_kv(const void* k, const void* v, const void* dout,
-                              const sla_block_lists& cols, const float* o_lin, float* dk,
-                              float* dv, float* dproj, const Geom& g, void* scratch,
-                              int32_t* status, cudaStream_t s);
+// 2. between the dq and dkdv launches: dH_j, dz_j from dH^M, dz^M (the
+//    indicator GEMM over the column lists), and the pointers for the fused
+//    key side
+cudaError_t launch_lin_bwd_gather(const sla_block_lists& cols, const Geom& g, void* scratch,
+                                  int32_t* status, cudaStream_t s, LinBwdKIn* lin);
+// 3. dW = O_lin^T dO (zero without a linear branch)
+cudaError_t launch_lin_bwd_dw(const void* dout, const float* o_lin, float* dproj, const Geom& g,
+                              void* scratch, int32_t* status, cudaStream_t s);
 
 // backward
 cudaError_t launch_bwd_prep(const void* dout, const float* o_s,

@@ -20,14 +20,13 @@
 // arithmetic; g, dnum, dH^M and dH go through bf16 once as MMA operands.
 //
 // Kernels here (all waits bounded; timeouts set the status word):
-//   delta_kernel         Delta_t = dO_t . O_s[t]                (HBM-bound)
-//   dw_tc_kernel         dW partials, persistent over 128-token tiles
-//   lin_bwd_kv_tc_kernel one CTA per key block that is marginal somewhere,
-//                        working transposed (TMEM lane = channel, column =
-//                        token)
+//   delta_kernel   Delta_t = dO_t . O_s[t]                (HBM-bound)
+//   dw_tc_kernel   dW partials, persistent over 128-token tiles
 // The query side (g, dnum, dq, dH^M, dz^M) runs in the epilogue of the
-// critical branch's dq kernel (attn_bwd_tc.cu), where Q, dO and dQ already
-// sit on chip.
+// critical branch's dq kernel and the key side (dk, dv) in the epilogue of
+// its dkdv kernel (attn_bwd_tc.cu), where the operands already sit on chip;
+// between the two, the indicator GEMM over the column lists sums dH^M, dz^M
+// into dH_j, dz_j.
 #include <algorithm>
 
 #include "common.cuh"
@@ -185,114 +184,6 @@ __global__ void dw_sum_kernel(const float* __restrict__ part, float* __restrict_
   dproj[i] = s;
 }
 
-// ---------------------------------------------------------------------------
-// Key side: one CTA (128 threads, thread = channel) per (key block j, bh)
-// that is marginal for some query block.
-//   dv^T    = dH^T phi(K)^T   (M = 128 channels c, N = BK tokens, K = 128 a)
-//   dphi^T  = dH V^T          (M = 128 channels a, N = BK tokens, K = 128 c)
-//   dv_u += dv^T[:, u];  dk_u += (dphi^T[:, u] + dz_j) o phi'(k_u)
-template <int BK>
-__global__ void __launch_bounds__(128) lin_bwd_kv_tc_kernel(
-    const __grid_constant__ CUtensorMap tmDH, const __grid_constant__ CUtensorMap tmK,
-    const __grid_constant__ CUtensorMap tmV, const float* __restrict__ dzb,
-    const int32_t* __restrict__ marg_cnt, const __nv_bfloat16* __restrict__ k,
-    float* __restrict__ dk, float* __restrict__ dv, int N, int nkb, int nqb, int32_t* status) {
-  constexpr uint32_t kKC = BK * 128;
-  constexpr uint32_t offDH = 0, offK = 32768, offV = offK + 2 * kKC;
-  constexpr uint32_t offBar = offV + 2 * kKC;
-  constexpr uint32_t kCols = BK == 64 ? 128 : 256;  // dv^T at 0, dphi^T at BK
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = align1k(smem_raw);
-  const uint32_t sb = smem_u32(base);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + offBar);
-  const uint32_t b_tma = smem_u32(&bars[0]), b_mma = smem_u32(&bars[1]);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(&bars[2]);
-  const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid / 32;
-  const int list_row = bh * nkb + j;
-  if (min(max(marg_cnt[list_row], 0), nqb) == 0) return;  // never marginal: nothing to add
-  const int u0 = j * BK, valid = min(BK, N - u0);
-  if (tid == 0) {
-    mbar_init(b_tma, 1);
-    mbar_init(b_mma, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) tmem_alloc(smem_u32(tslot), kCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const int c = tid;
-  if (tid == 0) {
-    mbar_expect_tx(b_tma, 32768 + 4 * kKC);
-    const int hrow = list_row * kLD;
-    tma_load_2d(sb + offDH, &tmDH, 0, hrow, b_tma);
-    tma_load_2d(sb + offDH + 16384, &tmDH, 64, hrow, b_tma);
-    tma_load_3d(sb + offK, &tmK, 0, u0, bh, b_tma);
-    tma_load_3d(sb + offK + kKC, &tmK, 64, u0, bh, b_tma);
-    tma_load_3d(sb + offV, &tmV, 0, u0, bh, b_tma);
-    tma_load_3d(sb + offV + kKC, &tmV, 64, u0, bh, b_tma);
-  }
-  const float dzc = dzb[static_cast<i64>(list_row) * kLD + c];
-  bool ok = __syncthreads_and(wait_bounded(b_tma, 0, status, kLbTimeout));
-  if (ok) {
-    for (int x = tid; x < BK * 16; x += 128) {  // phi(K) in place, rows past N zero
-      const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
-      uint4* p = reinterpret_cast<uint4*>(base + offK + chunk * kKC + sw128(row, u));
-      *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idv = idesc_bf16(128, BK, 1, 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma(tmem, sdesc(sb + offDH + kk * 2048, 16384, 1024),
-               sdesc(sb + offK + (kk >> 2) * kKC + (kk & 3) * 32, 16, 1024), idv, kk > 0);
-      constexpr uint32_t idp = idesc_bf16(128, BK, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma(tmem + BK, sdesc(sb + offDH + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-               sdesc(sb + offV + (kk >> 2) * kKC + (kk & 3) * 32, 16, 1024), idp, kk > 0);
-      tc_commit(b_mma);
-    }
-    ok = __syncthreads_and(wait_bounded(b_mma, 0, status, kLbTimeout));
-  }
-  if (ok) {
-    tc_fence_after();
-#pragma unroll
-    for (int tt = 0; tt < BK; tt += 32) {
-      float a[32], b[32];
-      tmem_ld32(tmem + lane_off + tt, a);
-      tmem_ld32(tmem + BK + lane_off + tt, b);
-      tmem_wait_ld();
-      reg_fence<32>(a);
-      reg_fence<32>(b);
-#pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int u = tt + q;
-        if (u < valid) {
-          const i64 off = (static_cast<i64>(bh) * N + u0 + u) * kLD + c;
-          dv[off] += a[q];
-          dk[off] += (b[q] + dzc) * dphi(__bfloat162float(k[off]));
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (!ok) {
-    const long long t0 = clock64();
-    while (clock64() - t0 < 2000000) __nanosleep(1000);
-  }
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kCols);
-  }
-}
-
 template <typename F>
 cudaError_t lb_set_smem(F kern, size_t bytes) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -359,50 +250,29 @@ cudaError_t launch_lin_bwd_prepare(const void* k, const void* v, const float* pr
   return cudaSuccess;
 }
 
-cudaError_t launch_lin_bwd_kv(const void* k, const void* v, const void* dout,
-                              const sla_block_lists& cols, const float* o_lin, float* dk,
-                              float* dv, float* dproj, const Geom& g, void* scratch,
-                              int32_t* status, cudaStream_t s) {
+cudaError_t launch_lin_bwd_gather(const sla_block_lists& cols, const Geom& g, void* scratch,
+                                  int32_t* status, cudaStream_t s, LinBwdKIn* lin) {
   if (!lin_tc_supported(g)) return cudaErrorNotSupported;
   const LinBwdWs w = lin_bwd_ws(g);
   char* sc = static_cast<char*>(scratch);
-  const uint64_t BH = g.BH, N = g.N, nkb = g.nkb;
-  cudaError_t e;
-  if (g.linear) {
-    // dH_j, dz_j: the indicator GEMM over the column lists (dH^M, dz^M were
-    // written by the dq kernel, zeros for query blocks without marginal sets)
-    if ((e = launch_list_gather(cols, g.BH, g.nkb, g.nqb, sc + w.dhm,
-                                reinterpret_cast<const float*>(sc + w.dzm), sc + w.dh,
-                                reinterpret_cast<float*>(sc + w.dz), sc + w.indt, w.ldt, status, s)) !=
-        cudaSuccess)
-      return e;
-    CUtensorMap mDH, mK, mV;
-    const uint64_t dq3[3] = {kLD, N, BH}, sq3[2] = {kLD * 2, N * kLD * 2};
-    const uint32_t boxk[3] = {64, static_cast<uint32_t>(g.bk), 1};
-    const uint64_t ddh[2] = {kLD, BH * nkb * kLD}, s2[1] = {kLD * 2};
-    const uint32_t box2[2] = {64, 128};
-    if (!encode_bf16_map(&mDH, sc + w.dh, 2, ddh, s2, box2) ||
-        !encode_bf16_map(&mK, k, 3, dq3, sq3, boxk) || !encode_bf16_map(&mV, v, 3, dq3, sq3, boxk))
-      return cudaErrorInvalidValue;
-    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
-    dim3 gk(g.nkb, g.BH);
-    const float* dz_p = reinterpret_cast<const float*>(sc + w.dz);
-    if (g.bk == 64) {
-      const size_t smem = 32768 + 4 * 64 * 128 + 64 + 1024;
-      if ((e = lb_set_smem(lin_bwd_kv_tc_kernel<64>, smem)) != cudaSuccess) return e;
-      lin_bwd_kv_tc_kernel<64><<<gk, 128, smem, s>>>(mDH, mK, mV, dz_p, cols.marg_cnt, kb, dk, dv, g.N,
-                                                     g.nkb, g.nqb, status);
-    } else {
-      const size_t smem = 32768 + 4 * 128 * 128 + 64 + 1024;
-      if ((e = lb_set_smem(lin_bwd_kv_tc_kernel<128>, smem)) != cudaSuccess) return e;
-      lin_bwd_kv_tc_kernel<128><<<gk, 128, smem, s>>>(mDH, mK, mV, dz_p, cols.marg_cnt, kb, dk, dv, g.N,
-                                                      g.nkb, g.nqb, status);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  // dW = O_lin^T dO (zero without a linear branch, where O_lin is zero)
+  // dH^M, dz^M were written by the dq kernel (zeros for query blocks
+  // without marginal sets)
+  cudaError_t e = launch_list_gather(cols, g.BH, g.nkb, g.nqb, sc + w.dhm,
+                                     reinterpret_cast<const float*>(sc + w.dzm), sc + w.dh,
+                                     reinterpret_cast<float*>(sc + w.dz), sc + w.indt, w.ldt, status, s);
+  if (e != cudaSuccess) return e;
+  lin->dh = sc + w.dh;
+  lin->dz = reinterpret_cast<const float*>(sc + w.dz);
+  lin->marg_cnt = cols.marg_cnt;
+  return cudaSuccess;
+}
+
+cudaError_t launch_lin_bwd_dw(const void* dout, const float* o_lin, float* dproj, const Geom& g,
+                              void* scratch, int32_t* status, cudaStream_t s) {
   if (!g.linear) return cudaMemsetAsync(dproj, 0, sizeof(float) * kLHElems, s);
-  const i64 R = static_cast<i64>(BH) * N;
+  const LinBwdWs w = lin_bwd_ws(g);
+  char* sc = static_cast<char*>(scratch);
+  const i64 R = static_cast<i64>(g.BH) * g.N;
   CUtensorMap mdO2;
   const uint64_t d2[2] = {kLD, static_cast<uint64_t>(R)}, s2[1] = {kLD * 2};
   const uint32_t box2[2] = {64, 128};
@@ -410,6 +280,7 @@ cudaError_t launch_lin_bwd_kv(const void* k, const void* v, const void* dout,
   const int parts = static_cast<int>(std::min<i64>(kDwParts, (R + 127) / 128));
   float* part = reinterpret_cast<float*>(sc + w.part);
   const size_t smem = 2 * kDwStage + 64 + 1024;
+  cudaError_t e;
   if ((e = lb_set_smem(dw_tc_kernel, smem)) != cudaSuccess) return e;
   dw_tc_kernel<<<parts, 128, smem, s>>>(mdO2, o_lin, part, R, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -419,18 +419,23 @@ sla_status sla_backward(const sla_params* p, const void* q, const void* k,
     if (linear)
       SLA_CUDA(sla::launch_lin_bwd_prepare(k, v, proj, *rows, o_lin, g, at<char>(ws, w.lin), status,
                                            s, &lin));
-    SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
-                                     at<char>(ws, w.plans), status, s, linear ? &lin : nullptr));
-    SLA_CUDA(sla::launch_lin_bwd_kv(k, v, dout, *cols, o_lin, dk, dv, dproj, g, at<char>(ws, w.lin),
-                                    status, s));
+    SLA_CUDA(sla::launch_attn_bwd_tc_dq(q, k, v, dout, lse, delta, *rows, *cols, dq, g,
+                                        at<char>(ws, w.plans), status, s, linear ? &lin : nullptr));
+    sla::LinBwdKIn link{};
+    if (linear) SLA_CUDA(sla::launch_lin_bwd_gather(*cols, g, at<char>(ws, w.lin), status, s, &link));
+    SLA_CUDA(sla::launch_attn_bwd_tc_dkdv(q, k, v, dout, lse, delta, dk, dv, g, at<char>(ws, w.plans),
+                                          status, s, linear ? &link : nullptr));
+    SLA_CUDA(sla::launch_lin_bwd_dw(dout, o_lin, dproj, g, at<char>(ws, w.lin), status, s));
     return SLA_OK;
   }
   float* gbuf = at<float>(ws, w.gbuf);
   float* dwp = at<float>(ws, w.dwp);
   SLA_CUDA(sla::launch_bwd_prep(dout, o_s, o_lin, proj, delta, gbuf, dwp, g, s));
   if (bwd_tc_attention(g)) {
-    SLA_CUDA(sla::launch_attn_bwd_tc(q, k, v, dout, lse, delta, *rows, *cols, dq, dk, dv, g,
-                                     at<char>(ws, w.plans), static_cast<int32_t*>(ws), s, nullptr));
+    SLA_CUDA(sla::launch_attn_bwd_tc_dq(q, k, v, dout, lse, delta, *rows, *cols, dq, g,
+                                        at<char>(ws, w.plans), static_cast<int32_t*>(ws), s, nullptr));
+    SLA_CUDA(sla::launch_attn_bwd_tc_dkdv(q, k, v, dout, lse, delta, dk, dv, g, at<char>(ws, w.plans),
+                                          static_cast<int32_t*>(ws), s, nullptr));
   } else {
     SLA_CUDA(sla::launch_attn_bwd_dq(q, k, v, dout, lse, delta, *rows, dq, g, s));
     SLA_CUDA(sla::launch_attn_bwd_dkdv(q, k, v, dout, lse, delta, *cols, dk, dv, g, s));
