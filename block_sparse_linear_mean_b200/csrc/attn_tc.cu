@@ -13,16 +13,24 @@
 //     (one block of 128 or two listed blocks of 64).  A row only attends to
 //     keys whose block is in its own query block's list (masked otherwise).
 //   * Warp 0 (one lane): TMA producer -- Q once, then K and V per key tile
-//     into a 2-stage ring, with the 3D tensor map [B*H, N, d] so rows past N
-//     read as zeros.
-//   * Warp 1 (one lane): MMA issuer -- S = Q K^T (M=128, N=128, K=d) into a
-//     double-buffered TMEM tile, O += P V (M=128, N=d, K=128) into TMEM.
-//   * Warps 2-5: one thread per query row -- tcgen05.ld of its S row, masking,
-//     online softmax in the exp2 domain with lazy rescaling (the running max
-//     is only moved when it grows by more than 2^8, which keeps P <= 256),
-//     P as bf16 into a 128B-swizzled shared-memory tile, and the epilogue
-//     O / l and LSE.  The row sum l accumulates the bf16-rounded P, the same
-//     weights the PV product uses.
+//     into two 3-stage rings, with the 3D tensor map [B*H, N, d] so rows past
+//     N read as zeros.
+//   * Warp 1 (one lane): MMA issuer -- S = Q K^T (M=128, N=128, K=d) into the
+//     TMEM buffer of the tile's parity, O_h += P V (M=128, N=d, K=128) with P
+//     read from TMEM.
+//   * Warps 2-9: two warpgroups that take alternate key tiles.  Warpgroup h
+//     owns the tiles of parity h, the S buffer h and the accumulator O_h; a
+//     thread holds one 128-key row of S -- tcgen05.ld, masking, online
+//     softmax in the exp2 domain, and P as bf16 pairs over its own S columns.
+//     No row statistic crosses warps inside the loop; (m_h, l_h, O_h) of the
+//     two warpgroups are merged once in the epilogue (O / l, LSE).  The two
+//     warps that share a TMEM lane quadrant -- and an SM sub-partition --
+//     work on different tiles, so one's exponentials overlap the other's
+//     loads and stores.  The running max lags a tile: P uses the max of the
+//     earlier tiles while the tile's max accumulates in the same pass, and a
+//     growth beyond 2^8 raises it on the next tile (P stays below 2^64
+//     meanwhile, far inside the fp32 and bf16 range; a larger jump redoes
+//     the tile exactly).
 // Every mbarrier wait is bounded: on expiry the CTA records SLA_ERR_TIMEOUT
 // in the status word, drains, frees its TMEM and returns.
 #include <cuda.h>
@@ -39,7 +47,7 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 3;
-constexpr int kSBuf = 3;  // S tiles in TMEM (P of a tile overwrites its S)
+constexpr int kSBuf = 2;  // S tiles in TMEM, one per warpgroup (P overwrites its S)
 // One pair in kPolyEvery of a full tile's exponentials is computed by a cubic
 // on the FMA pipe instead of the special-function unit (0: none).
 constexpr int kPolyEvery = 3;
@@ -48,6 +56,7 @@ constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softma
 constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr float kGuardLog2 = 64.0f;  // largest exponent of P the one-pass softmax accepts
 
 // ------------------------------------------------------------------ plan
 // One key-tile descriptor packs two 16-bit entries (the second only used for
@@ -141,8 +150,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   constexpr uint32_t offK = offQ + kQBytes;
   constexpr uint32_t offV = offK + kStages * kKBytes;
   constexpr uint32_t offOL = offK + 2 * kKBytes;       // O_lin (bf16) after the loop: K stage 2
-  constexpr uint32_t offRed = offV + kStages * kKBytes;  // [2 parity][2 halves][128] fp32
-  constexpr uint32_t offBar = offRed + 2 * 2 * 128 * 4;
+  // merge area of the epilogue ([m | l | den][2 warpgroups][128] fp32), in V
+  // stage 1, free once every P V product is done
+  constexpr uint32_t offX = offV + kKBytes;
+  constexpr uint32_t offBar = offV + kStages * kKBytes;
   constexpr uint32_t kUsed = offBar + 512;
   constexpr uint32_t idesc_qk = idesc_bf16(128, kTileN, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
@@ -159,15 +170,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto b_v_full = [&](int s) { return smem_u32(&bars[1 + kStages + s]); };
   auto b_k_empty = [&](int s) { return smem_u32(&bars[1 + 2 * kStages + s]); };
   auto b_v_empty = [&](int s) { return smem_u32(&bars[1 + 3 * kStages + s]); };
-  // per S buffer j = t % kSBuf: S(t) in TMEM, P(t) in TMEM (8 warps), P V of
-  // tile t done
-  auto b_s_full = [&](int j) { return smem_u32(&bars[kB0 + j]); };
-  auto b_p_full = [&](int j) { return smem_u32(&bars[kB0 + kSBuf + j]); };
-  auto b_pv_done = [&](int j) { return smem_u32(&bars[kB0 + 2 * kSBuf + j]); };
-  constexpr int kB1 = kB0 + 3 * kSBuf;
-  // partial row maxima exchanged between the two warps holding the same 32
-  // rows (one per column half): one barrier per (tile parity, lane quadrant)
-  auto b_red = [&](int b, int quad) { return smem_u32(&bars[kB1 + 9 + 4 * b + quad]); };
+  // per S buffer h (tiles of parity h): S(t) in TMEM, P(t) in TMEM (the four
+  // warps of warpgroup h)
+  auto b_s_full = [&](int h) { return smem_u32(&bars[kB0 + h]); };
+  auto b_p_full = [&](int h) { return smem_u32(&bars[kB0 + kSBuf + h]); };
+  constexpr int kB1 = kB0 + 2 * kSBuf;
   const uint32_t b_fin = smem_u32(&bars[kB1 + 0]);
   const uint32_t b_lin = smem_u32(&bars[kB1 + 1]);   // H^M and W tiles landed
   const uint32_t b_phiq = smem_u32(&bars[kB1 + 2]);  // phi(Q) written (8 warps)
@@ -175,15 +182,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t b_num = smem_u32(&bars[kB1 + 4]);   // phi(Q) H^M in TMEM
   const uint32_t b_olin = smem_u32(&bars[kB1 + 5]);  // O_lin (bf16) in shared memory (8 warps)
   const uint32_t b_lout = smem_u32(&bars[kB1 + 6]);  // O_lin W in TMEM
-  // every P V product done (single use).  The producer cannot wait on
-  // pv_done for this: the completion before the last one on the same
-  // barrier may still be pending, and a parity wait would then take the
-  // older phase for the newer one.
+  // every P V product done (single use): the producer's linear loads and
+  // the epilogue wait on it
   const uint32_t b_pv_last = smem_u32(&bars[kB1 + 7]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB1 + 17]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB1 + 18]);
-  static_assert((kB1 + 19) * 8 <= kUsed - offBar, "barrier block too small");
-  float* red = reinterpret_cast<float*>(base + offRed);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[kB1 + 8]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[kB1 + 9]);
+  static_assert((kB1 + 10) * 8 <= kUsed - offBar, "barrier block too small");
+  float* xch = reinterpret_cast<float*>(base + offX);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int tile = blockIdx.x;
@@ -219,11 +224,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     for (int j = 0; j < kSBuf; ++j) {
       mbar_init(b_s_full(j), 1);
-      mbar_init(b_p_full(j), kSoftmaxWarps);
-      mbar_init(b_pv_done(j), 1);
+      mbar_init(b_p_full(j), kSoftmaxWarps / 2);
     }
-    for (int b = 0; b < 2; ++b)
-      for (int q = 0; q < 4; ++q) mbar_init(b_red(b, q), 2);
     mbar_init(b_fin, kSoftmaxWarps);
     mbar_init(b_lin, 1);
     mbar_init(b_phiq, kSoftmaxWarps);
@@ -235,7 +237,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // TMEM: 512 columns (S0 | S1 | S2 | O)
+  if (warp == 1) {  // TMEM: 512 columns (S0 | S1 | O_0 | O_1)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -244,13 +246,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // columns: S of tile t at 128 (t % kSBuf), O at 384.  The bf16 P of tile t
-  // (two keys per column) overwrites its own S: the column half h puts its
-  // 32 P columns at 64 h, columns that only its own threads read.
-  // Addresses are computed, not indexed from an array, so none goes through
-  // local memory.
+  // columns: S of tile t at 128 (t % 2), O_h at 256 + 128 h.  The bf16 P of
+  // tile t (two keys per column) overwrites the last 64 columns of its own
+  // S, which only the warp holding those rows reads.  Addresses are computed,
+  // not indexed from an array, so none goes through local memory.
   auto tS = [&](int j) { return tmem + 128u * static_cast<uint32_t>(j); };
-  const uint32_t tO = tmem + 384;
+  auto tO = [&](int h) { return tmem + 256u + 128u * static_cast<uint32_t>(h); };
 
   auto give_up = [&]() {
     *abort_flag = 1;
@@ -338,13 +339,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t dQ = sdesc(sb + offQ, 16, 1024);
       const uint64_t dK0 = sdesc(sb + offK, 16, 1024);
       const uint64_t dV0 = sdesc(sb + offV, 16384, 1024);
-      auto issue_s = [&](int t) -> bool {
-        const int s = t % kStages, j = t % kSBuf;
-        if (!wait(b_k_full(s), (t / kStages) & 1)) return false;
-        // S(t) takes the buffer of tile t - kSBuf: that tile's softmax is done
-        // (its P V was issued after its P arrived, before this call) and the
-        // tensor pipe reads that P before this MMA overwrites it (it runs in
-        // issue order)
+      // S(t) takes the buffer of tile t - 2, whose P V was issued just before:
+      // the tensor pipe runs in issue order, so it reads that P before this
+      // MMA overwrites it.  The caller has waited for K(t).
+      auto issue_s = [&](int t) {
+        const int s = t % kStages, j = t & 1;
         tc_fence_after();
         const uint64_t dK = sdesc_add(dK0, s * kKBytes);
 #pragma unroll
@@ -354,31 +353,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         tc_commit(b_s_full(j));
         tc_commit(b_k_empty(s));
-        return true;
       };
-      auto issue_pv = [&](int t) -> bool {
-        const int s = t % kStages, j = t % kSBuf;
-        if (!wait(b_p_full(j), (t / kSBuf) & 1)) return false;
-        if (!wait(b_v_full(s), (t / kStages) & 1)) return false;
+      // the caller has waited for P(t) and V(t)
+      auto issue_pv = [&](int t) {
+        const int s = t % kStages, j = t & 1;
         tc_fence_after();
         const uint64_t dV = sdesc_add(dV0, s * kKBytes);
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
-          tc_mma_ts(tO, tS(j) + 64 * (kk / 4) + (kk % 4) * 8, sdesc_add(dV, kk * 2048), idesc_pv,
-                    (t > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tO(j), tS(j) + 64 + kk * 8, sdesc_add(dV, kk * 2048), idesc_pv, (t > 1 || kk > 0) ? 1u : 0u);
         tc_commit(b_v_empty(s));
-        tc_commit(b_pv_done(j));
-        return true;
       };
-      // S(t + 2) is issued before the wait for P(t) (its buffer was last
-      // read by P V of tile t - 1, issued in the previous round), so the
-      // tensor pipe computes it while the softmax works on tile t, and a
-      // softmax warp that finishes a tile finds the next S already done
-      if (ok) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
+      // S of the next tile of the same parity follows each P V product;
+      // the other warpgroup's tile keeps the tensor pipe busy meanwhile.
+      // The commit of S(t + 2) also tells that warpgroup that P V of tile t
+      // is complete (commits track every earlier MMA), which its rescale of
+      // O relies on.  The operands of the next two products are waited for
+      // before P(t): they are almost always there already, and the wait for
+      // the softmax is then the only one between P(t) and the tensor pipe.
+      for (int t = 0; ok && t < 2 && t < T; ++t) {
+        ok = wait(b_k_full(t), 0);
+        if (ok) issue_s(t);
+      }
       for (int t = 0; ok && t < T; ++t) {
-        if (t + 2 < T) ok = issue_s(t + 2);
-        if (ok) ok = issue_pv(t);
+        ok = wait(b_v_full(t % kStages), (t / kStages) & 1);
+        if (ok && t + 2 < T) ok = wait(b_k_full((t + 2) % kStages), ((t + 2) / kStages) & 1);
+        if (ok) ok = wait(b_p_full(t & 1), (t >> 1) & 1);
+        if (!ok) break;
+        issue_pv(t);
+        if (t + 2 < T) issue_s(t + 2);
       }
       if (ok) tc_commit(b_pv_last);
     }
@@ -416,153 +419,195 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else {
     // ---------------------------------------------------------- softmax
-    // Two warpgroups; thread (h, r) owns columns [64h, 64h + 64) of query
-    // row r and O columns [h*D/2, (h+1)*D/2).  The two halves of a row
-    // exchange their partial maxima through shared memory every tile, so
-    // both keep the same running max and rescale decisions.
-    const int h = (warp - 2) >> 2;        // column half
+    // Warpgroup h takes the key tiles t = h, h + 2, ...; thread (h, r) holds
+    // row r of those tiles and keeps its own running max, sum and O_h.
+    const int h = (warp - 2) >> 2;        // tile parity = S buffer = O accumulator
     const int quad = warp & 3;            // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;       // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t rflag = BQ == 128 ? 3u : (r < 64 ? 1u : 2u);
     const unsigned full = 0xffffffffu;
-    float m_ref = -INFINITY, l = 0.f;
+    const uint32_t tSh = tS(h) + lane_off, tOh = tO(h) + lane_off;
+    // running max (log2 domain), a raise of it due on the next tile, sum
+    float m_ref = -INFINITY, pend = -INFINITY, l = 0.f;
     bool ok = true;
-    // the plan word of the next tile is fetched a tile ahead: a global load
-    // on the path from one tile to the next would stall every warp
-    uint32_t desc_next = T > 0 ? ptiles[0] : 0u;
-    for (int t = 0; ok && t < T; ++t) {
-      const int b = t & 1, j = t % kSBuf;
-      const uint32_t desc = desc_next;
-      if (t + 1 < T) desc_next = ptiles[t + 1];
-      // this thread's 64 keys: entry h of a tile of two 64-blocks, or half h
-      // of one 128-block
-      const uint32_t ent = BK == 64 ? (desc >> (16 * h)) & 0xFFFFu : desc & 0xFFFFu;
+    // valid keys of row r among the 64 keys from blk * BK + off of entry ent
+    auto nvalid = [&](uint32_t ent, int off) -> int {
       const int blk = ent & 0x1FFF;
       const bool member = (ent & kPresent) && (((ent >> 13) & 3u) & rflag);
-      const int kvalid = member ? max(0, min(64, N - blk * BK - (BK == 128 ? h * 64 : 0))) : 0;
-      if (!__all_sync(full, wait(b_s_full(j), (t / kSBuf) & 1))) { ok = false; break; }
+      return member ? max(0, min(64, N - blk * BK - off)) : 0;
+    };
+    // the plan word of the next tile is fetched a tile ahead: a global load
+    // on the path from one tile to the next would stall every warp
+    uint32_t desc_next = h < T ? ptiles[h] : 0u;
+    for (int t = h; ok && t < T; t += 2) {
+      const uint32_t use = static_cast<uint32_t>(t) >> 1;  // earlier uses of buffer h
+      const uint32_t desc = desc_next;
+      if (t + 2 < T) desc_next = ptiles[t + 2];
+      // keys [0, 64) and [64, 128) of the tile: the two entries of a pair of
+      // 64-blocks, or the two halves of one 128-block
+      const int kv0 = nvalid(desc & 0xFFFFu, 0);
+      const int kv1 = BK == 64 ? nvalid(desc >> 16, 0) : nvalid(desc & 0xFFFFu, 64);
+      if (!__all_sync(full, wait(b_s_full(h), use & 1))) { ok = false; break; }
       tc_fence_after();
+      // The row is read in two halves of 64 keys, so that 64 scores are live
+      // at a time.  P (key k at column 64 + k / 2) goes over the columns of
+      // keys 64-127 once every score of the tile has been read.
       float s[64];
-      tmem_ld32(tS(j) + lane_off + h * 64, s);
-      tmem_ld32(tS(j) + lane_off + h * 64 + 32, s + 32);
-      tmem_wait_ld();
-      reg_fence<64>(s);
-      // partial max of the raw scores over this thread's valid keys (four
-      // independent three-input chains)
-      float mx = -INFINITY;
-      if (kvalid == 64) {
-        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+      auto load_half = [&](int e) {
+        tmem_ld32(tSh + 64 * e, s);
+        tmem_ld32(tSh + 64 * e + 32, s + 32);
+        tmem_wait_ld();
+        reg_fence<64>(s);
+      };
+      // O_h *= alpha (warp-wide TMEM access; alpha = 1 on rows that keep
+      // their scale).  No wait is needed: S(t) has completed, and its commit
+      // followed P V of tile t - 2, the last product into O_h.
+      auto rescale_o = [&](float alpha) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          a0 = max3(a0, s[c], s[c + 1]);
-          a1 = max3(a1, s[c + 2], s[c + 3]);
-          a2 = max3(a2, s[c + 4], s[c + 5]);
-          a3 = max3(a3, s[c + 6], s[c + 7]);
-        }
-        mx = max3(a0, a1, fmaxf(a2, a3));
-      } else if (kvalid > 0) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) mx = c < kvalid ? fmaxf(mx, s[c]) : mx;
-      }
-      red[(b * 2 + h) * 128 + r] = mx;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_red(b, quad));
-      if (!__all_sync(full, wait(b_red(b, quad), (t >> 1) & 1))) { ok = false; break; }
-      const float mo = red[(b * 2 + (h ^ 1)) * 128 + r];
-      const float mraw = fmaxf(mx, mo);
-      // running max (scaled, log2 domain) with lazy rescale
-      bool rescale = false;
-      float alpha = 1.f;
-      if (mraw > -INFINITY) {
-        const float mt = mraw * scale_log2;
-        if (m_ref == -INFINITY) {
-          m_ref = mt;
-        } else if (mt > m_ref + kRescaleLog2) {
-          alpha = exp2f(m_ref - mt);
-          m_ref = mt;
-          l *= alpha;
-          rescale = true;
-        }
-      }
-      // P = 2^(s * scale_log2 - m_ref) rounded to bf16.  The row sum uses the
-      // rounded weights the MMA sees, so O / l is an exact convex
-      // combination of V rows.
-      uint32_t pk[32];
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_ref, -m_ref);
-      if (kvalid == 64) {
-        // every kPolyEvery-th pair of exponentials goes to the FMA pipe
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
-          const float2 e = (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1)
-                               ? exp2_poly2(x)
-                               : make_float2(fast_exp2(x.x), fast_exp2(x.y));
-          pk[i] = pack_bf16x2(e.x, e.y);
-        }
-      } else if (kvalid > 0) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
-          pk[i] = pack_bf16x2(2 * i < kvalid ? fast_exp2(x.x) : 0.f,
-                              2 * i + 1 < kvalid ? fast_exp2(x.y) : 0.f);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        acc0 = add2(acc0, make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
-        acc1 = add2(acc1, make_float2(__uint_as_float(pk[i + 1] << 16), __uint_as_float(pk[i + 1] & 0xFFFF0000u)));
-        acc2 = add2(acc2, make_float2(__uint_as_float(pk[i + 2] << 16), __uint_as_float(pk[i + 2] & 0xFFFF0000u)));
-        acc3 = add2(acc3, make_float2(__uint_as_float(pk[i + 3] << 16), __uint_as_float(pk[i + 3] & 0xFFFF0000u)));
-      }
-      acc0 = add2(add2(acc0, acc1), add2(acc2, acc3));
-      l += acc0.x + acc0.y;
-      // P (bf16 pairs) over this half's own S columns: its 64 keys become
-      // columns [64h, 64h + 32) of the tile's buffer
-      tmem_st32u(tS(j) + lane_off + h * 64, pk);
-      // rescale this half of O (warp-wide TMEM access) once the previous
-      // P V is complete.  That parity wait cannot mistake an older phase:
-      // S(t) has completed and was issued after P V of tile t - 3, so P V of
-      // tile t - 4 (the barrier's previous use) is complete.
-      if (__any_sync(full, rescale)) {
-        if (t >= 1 && !__all_sync(full, wait(b_pv_done((t - 1) % kSBuf), ((t - 1) / kSBuf) & 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < DH; c += 32) {
+        for (int c = 0; c < D; c += 32) {
           float o[32];
-          tmem_ld32(tO + lane_off + h * DH + c, o);
+          tmem_ld32(tOh + c, o);
           tmem_wait_ld();
           reg_fence<32>(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tO + lane_off + h * DH + c, o);
+          tmem_st32(tOh + c, o);
         }
+      };
+      // a raise of the running max decided on the previous tile of this
+      // warpgroup takes effect now, P V of that tile being complete
+      if (__any_sync(full, pend > m_ref)) {
+        float alpha = 1.f;
+        if (pend > m_ref) {
+          alpha = exp2f(m_ref - pend);
+          m_ref = pend;
+          l *= alpha;
+        }
+        rescale_o(alpha);
       }
+      float2 acc0, acc1, acc2, acc3;
+      // exponentials of the loaded half (kv of its 64 keys valid) as bf16
+      // pairs into pk[0, 32), the sum of those rounded weights -- the ones
+      // P V uses, so O / l is a convex combination of V rows -- into acc;
+      // returns the max of the valid raw scores.  Every kPolyEvery-th pair of
+      // a full half goes to the FMA pipe.
+      auto half_exp = [&](int kv, uint32_t* pk) -> float {
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        const float2 nm2 = make_float2(-m_ref, -m_ref);
+        float mh = -INFINITY;
+        if (kv == 64) {
+          float a0 = -INFINITY, a1 = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i & 1) a1 = max3(a1, s[2 * i], s[2 * i + 1]);
+            else a0 = max3(a0, s[2 * i], s[2 * i + 1]);
+            const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
+            const float2 ex = (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1)
+                                  ? exp2_poly2(x)
+                                  : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            pk[i] = pack_bf16x2(ex.x, ex.y);
+            if (i % 4 == 0) add_bf16x2_f32(pk[i], acc0.x, acc0.y);
+            if (i % 4 == 1) add_bf16x2_f32(pk[i], acc1.x, acc1.y);
+            if (i % 4 == 2) add_bf16x2_f32(pk[i], acc2.x, acc2.y);
+            if (i % 4 == 3) add_bf16x2_f32(pk[i], acc3.x, acc3.y);
+          }
+          mh = fmaxf(a0, a1);
+        } else if (kv > 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int k = 2 * i;
+            mh = k < kv ? fmaxf(mh, s[k]) : mh;
+            mh = k + 1 < kv ? fmaxf(mh, s[k + 1]) : mh;
+            const float2 x = fma2(make_float2(s[k], s[k + 1]), sc2, nm2);
+            const float2 ex = make_float2(k < kv ? fast_exp2(x.x) : 0.f, k + 1 < kv ? fast_exp2(x.y) : 0.f);
+            pk[i] = pack_bf16x2(ex.x, ex.y);
+            if (i % 2 == 0) add_bf16x2_f32(pk[i], acc0.x, acc0.y);
+            else add_bf16x2_f32(pk[i], acc1.x, acc1.y);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        }
+        return mh;
+      };
+      // max of the valid raw scores of the loaded half
+      auto half_max = [&](int kv) -> float {
+        float mh = -INFINITY;
+        if (kv == 64) {
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            a0 = max3(a0, s[c], s[c + 1]);
+            a1 = max3(a1, s[c + 2], s[c + 3]);
+            a2 = max3(a2, s[c + 4], s[c + 5]);
+            a3 = max3(a3, s[c + 6], s[c + 7]);
+          }
+          mh = max3(a0, a1, fmaxf(a2, a3));
+        } else if (kv > 0) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) mh = c < kv ? fmaxf(mh, s[c]) : mh;
+        }
+        return mh;
+      };
+      // One pass: P with the running max of the earlier tiles while this
+      // tile's max accumulates.  Rows whose max grows by more than 2^8 raise
+      // the running max on the next tile; P stays below 2^kGuardLog2 (beyond
+      // that the tile is redone exactly), far inside the fp32 and bf16
+      // range.  The exact pass -- the first tile of a row, or a redo -- takes
+      // the tile's max first and raises the running max at once.
+      uint32_t pk[64];
+      bool exact = __any_sync(full, m_ref == -INFINITY);
+      for (int pass = 0; pass < 2; ++pass) {
+        if (exact) {
+          load_half(0);
+          float mx = half_max(kv0);
+          load_half(1);
+          mx = fmaxf(mx, half_max(kv1));
+          bool raise = false;
+          float alpha = 1.f;
+          if (mx > -INFINITY) {
+            const float mt = mx * scale_log2;
+            if (m_ref == -INFINITY) {
+              m_ref = mt;
+            } else if (mt > m_ref + kRescaleLog2) {
+              alpha = exp2f(m_ref - mt);
+              m_ref = mt;
+              l *= alpha;
+              raise = true;
+            }
+          }
+          if (__any_sync(full, raise)) rescale_o(alpha);
+        }
+        acc0 = acc1 = acc2 = acc3 = make_float2(0.f, 0.f);
+        load_half(1);
+        float mx = half_exp(kv1, pk + 32);
+        reg_fence_u<32>(pk + 32);  // keys 64-127 done before keys 0-63 load
+        load_half(0);
+        mx = fmaxf(mx, half_exp(kv0, pk));
+        const float mt = mx * scale_log2;
+        if (!exact && __any_sync(full, mt > m_ref + kGuardLog2)) {
+          exact = true;
+          continue;
+        }
+        tmem_st16u(tSh + 64, pk);
+        tmem_st16u(tSh + 80, pk + 16);
+        tmem_st16u(tSh + 96, pk + 32);
+        tmem_st16u(tSh + 112, pk + 48);
+        if (mt > m_ref + kRescaleLog2) pend = mt;  // (never after an exact pass)
+        break;
+      }
+      acc0 = add2(add2(acc0, acc1), add2(acc2, acc3));
+      l += acc0.x + acc0.y;
       tmem_wait_st();  // P (and any rescaled O) stored
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_p_full(j));
+      if (lane == 0) mbar_arrive(b_p_full(h));
     }
-    // epilogue: total row sum from both halves, O / l, LSE
-    const int fb = T & 1;  // red slot last used by tile T-2, read by all
-    red[(fb * 2 + h) * 128 + r] = l;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(b_fin);
-    bool fin = ok && __all_sync(full, wait(b_fin, 0));
-    const float ltot = fin ? l + red[(fb * 2 + (h ^ 1)) * 128 + r] : 0.f;
+    // epilogue.  Once every P V product is done O_0 and O_1 are final in
+    // TMEM, and Q, the K/V stages and the S columns are free.
     const int row = qt * kTileM + r;
     const i64 orow = (i64(bh) * N + row) * D + h * DH;
-    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-    // all P V products done: O final in TMEM, Q, the K/V stages and the S
-    // columns free
     // linear branch: this thread's half row of z^M (channels [64h, 64h + 64)),
     // fetched in one batch while the last P V products finish
     const bool second = BQ == 64 && r >= 64;
@@ -574,8 +619,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int i = 0; i < 16; ++i) z4[i] = __ldg(zp + i);
     }
-    if (fin && T > 0)
-      fin = __all_sync(full, wait(b_pv_done((T - 1) % kSBuf), ((T - 1) / kSBuf) & 1));
+    bool fin = ok && (T == 0 || __all_sync(full, wait(b_pv_last, 0)));
+    // merge the two warpgroups' (m, l) of row r; thread (h, r) then finishes
+    // O columns [h D/2, (h + 1) D/2) from both accumulators
+    xch[h * 128 + r] = m_ref;
+    xch[256 + h * 128 + r] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_fin);
+    fin = fin && __all_sync(full, wait(b_fin, 0));
+    const float m_o = fin ? xch[(h ^ 1) * 128 + r] : -INFINITY;
+    const float l_o = fin ? xch[256 + (h ^ 1) * 128 + r] : 0.f;
+    const float mt = fmaxf(m_ref, m_o);
+    const float f_s = m_ref > -INFINITY ? exp2f(m_ref - mt) : 0.f;
+    const float f_o = m_o > -INFINITY ? exp2f(m_o - mt) : 0.f;
+    const float ltot = fin ? l * f_s + l_o * f_o : 0.f;
+    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+    const float w0 = (h == 0 ? f_s : f_o) * inv, w1 = (h == 0 ? f_o : f_s) * inv;
     bool lin_ok = false;
     if (D == 128 && lin && fin) {  // (never taken for d = 64: lin is false)
       // phi(Q) in place (this thread: row r, channels [64h, 64h + 64)), and
@@ -600,8 +659,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           *p = val;
         }
         dpart += dpart2;
-        const int db = fb ^ 1;  // slot of tile T-1, read by all before b_fin
-        red[(db * 2 + h) * 128 + r] = dpart;
+        xch[512 + h * 128 + r] = dpart;
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -609,7 +667,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         lin_ok = __all_sync(full, wait(b_den, 0));
       }
       float den = 0.f;
-      if (lin_ok) den = dpart + red[((fb ^ 1) * 2 + (h ^ 1)) * 128 + r];
+      if (lin_ok) den = dpart + xch[512 + (h ^ 1) * 128 + r];
       if (lin_ok) lin_ok = __all_sync(full, wait(b_num, 0));
       if (lin_ok) {
         // O_lin = phi(Q) H^M / den -> o_lin (fp32, optional) and bf16 into K
@@ -651,12 +709,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
     for (int c = 0; c < DH; c += 32) {
       float o[32];
-      if (fin && T > 0) {
-        tmem_ld32(tO + lane_off + h * DH + c, o);
+      if (fin && T > 1) {
+        float o1[32];
+        tmem_ld32(tO(0) + lane_off + h * DH + c, o);
+        tmem_ld32(tO(1) + lane_off + h * DH + c, o1);
+        tmem_wait_ld();
+        reg_fence<32>(o);
+        reg_fence<32>(o1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = o[i] * w0 + o1[i] * w1;
+      } else if (fin && T > 0) {  // one tile: warpgroup 1 had none
+        tmem_ld32(tO(0) + lane_off + h * DH + c, o);
         tmem_wait_ld();
         reg_fence<32>(o);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] *= inv;
+        for (int i = 0; i < 32; ++i) o[i] *= w0;
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -685,7 +752,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
     if (row < N && h == 0)
-      ep.lse[i64(bh) * N + row] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
+      ep.lse[i64(bh) * N + row] = ltot > 0.f ? (mt + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
   }
 
   // teardown: on an abort let in-flight copies and MMAs drain (bounded)

@@ -153,6 +153,14 @@ __device__ __forceinline__ void reg_fence(float* v) {
 #pragma unroll
   for (int i = 0; i < K; ++i) asm volatile("" : "+f"(v[i]));
 }
+// Same for 32-bit integer registers: values computed before it stay computed
+// before any later volatile asm (a TMEM load, say), bounding how many
+// registers are live across it.
+template <int K>
+__device__ __forceinline__ void reg_fence_u(uint32_t* v) {
+#pragma unroll
+  for (int i = 0; i < K; ++i) asm volatile("" : "+r"(v[i]));
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 2^x with the hardware approximation (ex2.approx, flush-to-zero): relative
@@ -197,6 +205,14 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
   return r;
 }
+// a += low bf16 of v, b += high bf16 of v, in fp32 (mixed-precision add):
+// sums of bf16-rounded values without unpacking them first.
+__device__ __forceinline__ void add_bf16x2_f32(uint32_t v, float& a, float& b) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "r"(v));
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -222,8 +238,12 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                   make_float2(0.2426111251115799f, 0.2426111251115799f));
   p = fma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
   p = fma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+  // j sits in the low bits of t: p + t * 2^23 (mod 2^32) adds j to p's
+  // exponent in one multiply-add
+  uint32_t rx, ry;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(p.x)));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(p.y)));
+  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 // A descriptor advanced by `bytes` (a multiple of 16): the start address
