@@ -43,8 +43,11 @@ constexpr int kBwdStages = 4;
 constexpr uint32_t kBwdSmemRequest = 232448;
 constexpr uint32_t kBwdTmemCols = 512;
 // One pair in kBwdPolyEvery of a step's exponentials is computed by the
-// FMA-pipe cubic instead of the special-function unit.
-constexpr int kBwdPolyEvery = 3;
+// FMA-pipe cubic instead of the special-function unit (0: none).  The
+// elementwise warps are bound by latency, not by the special-function unit,
+// so the cubic's extra instructions cost more than they save.
+constexpr int kBwdPolyEvery = 0;
+constexpr int kBwdPolyStep = kBwdPolyEvery > 0 ? kBwdPolyEvery : 1;
 
 // A 64-row step of a plan word: entry e of a word of two 64-blocks, or half
 // e of one 128-block (skipped when it starts at or past N).
@@ -437,7 +440,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), c2, nl2);
-            float2 p = (kBwdPolyEvery > 0 && i % kBwdPolyEvery == kBwdPolyEvery - 1)
+            float2 p = (kBwdPolyEvery > 0 && i % kBwdPolyStep == kBwdPolyEvery - 1)
                            ? exp2_poly2(x)
                            : make_float2(fast_exp2(x.x), fast_exp2(x.y));
             if (kvalid < 32) {
@@ -960,7 +963,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           const float2 nl2 = *reinterpret_cast<const float2*>(nl + 2 * i);
           const float2 nd2 = *reinterpret_cast<const float2*>(nl + 64 + 2 * i);
           const float2 x = fma2(make_float2(sv[2 * i], sv[2 * i + 1]), c2, nl2);
-          float2 p = (kBwdPolyEvery > 0 && i % kBwdPolyEvery == kBwdPolyEvery - 1)
+          float2 p = (kBwdPolyEvery > 0 && i % kBwdPolyStep == kBwdPolyEvery - 1)
                          ? exp2_poly2(x)
                          : make_float2(fast_exp2(x.x), fast_exp2(x.y));
           if (!active) p = make_float2(0.f, 0.f);

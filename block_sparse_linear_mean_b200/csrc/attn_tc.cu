@@ -49,8 +49,11 @@ constexpr int kTileN = 128;
 constexpr int kStages = 3;
 constexpr int kSBuf = 2;  // S tiles in TMEM, one per warpgroup (P overwrites its S)
 // One pair in kPolyEvery of a full tile's exponentials is computed by a cubic
-// on the FMA pipe instead of the special-function unit (0: none).
-constexpr int kPolyEvery = 3;
+// on the FMA pipe instead of the special-function unit (0: none).  Here the
+// softmax warp is bound by latency rather than by the special-function
+// unit, and the cubic's extra instructions cost more than they save.
+constexpr int kPolyEvery = 0;
+constexpr int kPolyStep = kPolyEvery > 0 ? kPolyEvery : 1;
 constexpr int kSoftmaxWarps = 8;                 // two warpgroups
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softmax
 constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
@@ -503,7 +506,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (i & 1) a1 = max3(a1, s[2 * i], s[2 * i + 1]);
             else a0 = max3(a0, s[2 * i], s[2 * i + 1]);
             const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
-            const float2 ex = (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1)
+            const float2 ex = (kPolyEvery > 0 && i % kPolyStep == kPolyEvery - 1)
                                   ? exp2_poly2(x)
                                   : make_float2(fast_exp2(x.x), fast_exp2(x.y));
             pk[i] = pack_bf16x2(ex.x, ex.y);

@@ -253,7 +253,9 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 // cost to one 64-bit add; rebuilding a descriptor per MMA costs the issuing
 // thread more than the MMA itself takes on the tensor core.
 __device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
-  return desc + static_cast<uint64_t>(bytes >> 4);
+  // low word only: one 32-bit add (the high word cannot change)
+  const uint32_t lo = static_cast<uint32_t>(desc) + (bytes >> 4);
+  return (desc & 0xFFFFFFFF00000000ull) | lo;
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
