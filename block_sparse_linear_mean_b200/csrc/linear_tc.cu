@@ -181,102 +181,140 @@ __global__ void __launch_bounds__(128) indicator_kernel(sla_block_lists rows,
 }
 
 // 2b. Gather GEMM: HM[bh] (Nqb x 16384) = Ind[bh] (Nqb x ld) @ H[bh] (ld x 16384).
-//     CTA tile 128 x 256, K step 64, 4-stage TMA ring; warp 0 loads, warp 1
-//     issues tcgen05.mma (A K-major, B MN-major), warps 2-5 drain TMEM into a
-//     swizzled bf16 tile that one TMA store writes out.
-constexpr int kGStages = 4;
+//     Persistent: one CTA per SM walks output tiles of 128 x 256 (consecutive
+//     tiles share their H columns, so the CTAs working at one time read each
+//     H tile from L2 after the first).  K step 64, 3-stage TMA ring; warp 0
+//     loads, warp 1 issues tcgen05.mma (A K-major, B MN-major) into one of
+//     two TMEM accumulators, warps 2-5 drain the other into a swizzled bf16
+//     tile that TMA stores write out -- a tile's epilogue overlaps the next
+//     tile's products.
+constexpr int kGStages = 3;
 constexpr uint32_t kGA = 16384, kGB = 32768, kGStage = kGA + kGB;
+constexpr uint32_t kGStaging = kGStages * kGStage;       // 64 KB bf16 output tile
+constexpr uint32_t kGBars = kGStaging + 65536;
+constexpr size_t kGSmem = kGBars + 256 + 1024;
 
 __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const __grid_constant__ CUtensorMap tmC, int ksteps, int32_t* status) {
+    const __grid_constant__ CUtensorMap tmC, int ksteps, int tiles_m, int tiles_n, int ntiles,
+    int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const uint32_t sb = smem_u32(base);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kGStages * kGStage);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kGBars);
   auto b_full = [&](int s) { return smem_u32(&bars[s]); };
   auto b_empty = [&](int s) { return smem_u32(&bars[kGStages + s]); };
-  const uint32_t b_acc = smem_u32(&bars[2 * kGStages]);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(&bars[2 * kGStages + 1]);
-  const int n0 = blockIdx.x * 256, m0 = blockIdx.y * 128, bh = blockIdx.z;
+  auto b_acc_full = [&](int a) { return smem_u32(&bars[2 * kGStages + a]); };
+  auto b_acc_empty = [&](int a) { return smem_u32(&bars[2 * kGStages + 2 + a]); };
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(&bars[2 * kGStages + 4]);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGStages; ++s) { mbar_init(b_full(s), 1); mbar_init(b_empty(s), 1); }
-    mbar_init(b_acc, 1);
+    for (int a = 0; a < 2; ++a) { mbar_init(b_acc_full(a), 1); mbar_init(b_acc_empty(a), 4); }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) tmem_alloc(smem_u32(tslot), 256);
+  if (warp == 1) tmem_alloc(smem_u32(tslot), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // tile -> (m, n, bh), m fastest
+  auto coords = [&](int t, int& m0, int& n0, int& bh) {
+    const int per = tiles_m * tiles_n;
+    bh = t / per;
+    const int r = t - bh * per;
+    n0 = (r / tiles_m) * 256;
+    m0 = (r % tiles_m) * 128;
+  };
   bool ok = true;
   if (warp == 0 && lane == 0) {
-    for (int ks = 0; ks < ksteps && ok; ++ks) {
-      const int s = ks % kGStages;
-      if (ks >= kGStages) ok = wait_bounded(b_empty(s), ((ks / kGStages) & 1) ^ 1, status, kTimeout);
-      if (!ok) break;
-      const uint32_t st = sb + s * kGStage;
-      mbar_expect_tx(b_full(s), kGStage);
-      tma_load_3d(st, &tmA, ks * 64, m0, bh, b_full(s));
+    int g = 0;  // K steps loaded so far (ring position)
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      int m0, n0, bh;
+      coords(t, m0, n0, bh);
+      for (int ks = 0; ks < ksteps && ok; ++ks, ++g) {
+        const int s = g % kGStages;
+        if (g >= kGStages) ok = wait_bounded(b_empty(s), ((g / kGStages) & 1) ^ 1, status, kTimeout);
+        if (!ok) break;
+        const uint32_t st = sb + s * kGStage;
+        mbar_expect_tx(b_full(s), kGStage);
+        tma_load_3d(st, &tmA, ks * 64, m0, bh, b_full(s));
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tma_load_3d(st + kGA + c * 8192, &tmB, n0 + c * 64, ks * 64, bh, b_full(s));
+        for (int c = 0; c < 4; ++c) tma_load_3d(st + kGA + c * 8192, &tmB, n0 + c * 64, ks * 64, bh, b_full(s));
+      }
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16(128, 256, 0, 1);
     const uint64_t dA = sdesc(sb, 16, 1024), dB = sdesc(sb + kGA, 8192, 1024);  // built once
-    for (int ks = 0; ks < ksteps && ok; ++ks) {
-      const int s = ks % kGStages;
-      ok = wait_bounded(b_full(s), (ks / kGStages) & 1, status, kTimeout);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t so = s * kGStage;
+    int g = 0, it = 0;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+      const int a = it & 1;
+      // the epilogue has drained this accumulator (tile it - 2)
+      if (it >= 2) ok = wait_bounded(b_acc_empty(a), ((it >> 1) & 1) ^ 1, status, kTimeout);
+      for (int ks = 0; ks < ksteps && ok; ++ks, ++g) {
+        const int s = g % kGStages;
+        ok = wait_bounded(b_full(s), (g / kGStages) & 1, status, kTimeout);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t so = s * kGStage;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        tc_mma(tmem, sdesc_add(dA, so + kk * 32), sdesc_add(dB, so + kk * 2048), idesc,
-               (ks > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(b_empty(s));
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma(tmem + 256 * a, sdesc_add(dA, so + kk * 32), sdesc_add(dB, so + kk * 2048), idesc,
+                 (ks > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(b_empty(s));
+      }
+      if (ok) tc_commit(b_acc_full(a));
     }
-    if (ok) tc_commit(b_acc);
-  }
-  __syncthreads();  // every role has issued all it will issue
-  if (warp >= 2) ok = wait_bounded(b_acc, 0, status, kTimeout);
-  ok = __syncthreads_and(ok);
-  if (ok && warp >= 2) {
-    tc_fence_after();
+  } else if (warp >= 2) {
     const int quad = warp & 3, r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+      const int a = it & 1;
+      int m0, n0, bh;
+      coords(t, m0, n0, bh);
+      ok = wait_bounded(b_acc_full(a), (it >> 1) & 1, status, kTimeout);
+      // the previous tile's stores have read the staging tile
+      if (threadIdx.x == 64) tma_store_wait_read();
+      ok = bar_sync_and(1, 128, ok);  // all four warps take the same branch
+      if (!ok) break;
+      tc_fence_after();
 #pragma unroll
-    for (int c0 = 0; c0 < 256; c0 += 32) {
-      float v[32];
-      tmem_ld32(tmem + lane_off + c0, v);
-      tmem_wait_ld();
-      reg_fence<32>(v);
-      uint8_t* ch = base + (c0 >> 6) * 16384;  // staging: 4 chunks of [128 rows][64 cols]
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + 256 * a + lane_off + c0, v);
+        tmem_wait_ld();
+        reg_fence<32>(v);
+        uint8_t* ch = base + kGStaging + (c0 >> 6) * 16384;  // 4 chunks of [128 rows][64 cols]
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(ch + sw128(r, ((c0 & 63) >> 3) + q)) =
-            make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(ch + sw128(r, ((c0 & 63) >> 3) + q)) =
+              make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+      }
+      // accumulator free for tile it + 2
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_acc_empty(a));
+      fence_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 64) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tma_store_3d(&tmC, sb + kGStaging + c * 16384, n0 + c * 64, m0, bh);
+        tma_store_commit();
+      }
     }
-    fence_async_smem();
-  }
-  __syncthreads();
-  if (ok && threadIdx.x == 0) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tma_store_3d(&tmC, sb + c * 16384, n0 + c * 64, m0, bh);
-    tma_store_commit();
-    tma_store_wait_all();
+    if (threadIdx.x == 64) tma_store_wait_all();
   }
   tc_fence_before();
-  __syncthreads();
+  ok = __syncthreads_and(ok);
   if (!ok) {
     const long long t0 = clock64();
     while (clock64() - t0 < 2000000) __nanosleep(1000);
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -473,6 +511,26 @@ cudaError_t set_smem(F kern, size_t bytes) {
 
 }  // namespace
 
+// SMs of the current device (one persistent CTA each)
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
+}
+
+static cudaError_t launch_gather(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC,
+                                 int ld, int nrow, int BH, int32_t* status, cudaStream_t s) {
+  cudaError_t e;
+  if ((e = set_smem(gather_gemm_kernel, kGSmem)) != cudaSuccess) return e;
+  const int tiles_m = (nrow + 127) / 128, tiles_n = kHElems / 256;
+  const int ntiles = tiles_m * tiles_n * BH;
+  const int grid = std::min(ntiles, sm_count());
+  gather_gemm_kernel<<<grid, 192, kGSmem, s>>>(mA, mB, mC, ld / 64, tiles_m, tiles_n, ntiles, status);
+  return cudaGetLastError();
+}
+
 bool lin_tc_supported(const Geom& g) {
   return g.dtype == SLA_BF16 && g.d == kD && !(g.flags & SLA_FLAG_SIMT) && tma_available();
 }
@@ -513,11 +571,7 @@ cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, i
   if (!encode_bf16_map(&mA, indp, 3, da, sa, ba) || !encode_bf16_map(&mB, src_h, 3, db, sbt, bb) ||
       !encode_bf16_map(&mC, dst_h, 3, dc, sc2, bc))
     return cudaErrorInvalidValue;
-  const size_t smem = kGStages * kGStage + 256 + 1024;
-  if ((e = set_smem(gather_gemm_kernel, smem)) != cudaSuccess) return e;
-  dim3 grid(kHElems / 256, (nrow + 127) / 128, BH);
-  gather_gemm_kernel<<<grid, 192, smem, s>>>(mA, mB, mC, ld / 64, status);
-  return cudaGetLastError();
+  return launch_gather(mA, mB, mC, ld, nrow, BH, status, s);
 }
 
 cudaError_t launch_lin_tc_prepare(const void* k, const void* v, const float* proj,
@@ -601,13 +655,7 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
   // 2. indicator + gather GEMM
   indicator_kernel<<<g.BH * g.nqb, 128, 0, s>>>(rows, ind, zbuf, zmbuf, g.nqb, g.nkb, w.ld);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {
-    const size_t smem = kGStages * kGStage + 256 + 1024;
-    if ((e = set_smem(gather_gemm_kernel, smem)) != cudaSuccess) return e;
-    dim3 grid(kHElems / 256, (g.nqb + 127) / 128, g.BH);
-    gather_gemm_kernel<<<grid, 192, smem, s>>>(mA, mB, mC, w.ld / 64, status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+  if ((e = launch_gather(mA, mB, mC, w.ld, g.nqb, g.BH, status, s)) != cudaSuccess) return e;
   }  // prepare
   // 3-4. apply + combine
   if (apply) {
