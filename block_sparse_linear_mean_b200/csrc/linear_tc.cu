@@ -146,22 +146,27 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
 
 // ---------------------------------------------------------------------------
 // 2a. Marginal indicator Ind[bh, i, j] (bf16 0/1, row stride ld) from the
-//     CSR marginal lists, and z^M_i = sum of z_j over the list (fp32, list
-//     order): one CTA of 128 threads (one per channel) per query-block row.
+//     CSR marginal lists, and z^M_i = sum of z_j over the list (fp32): one
+//     CTA of 128 threads per query-block row.  Warp w sums the list entries
+//     e = w mod 4 (each lane four channels, one 16-byte load per entry, so a
+//     warp keeps several L2 reads in flight), and the four partial sums are
+//     added in a fixed order.
 __global__ void __launch_bounds__(128) indicator_kernel(sla_block_lists rows,
                                                         uint16_t* __restrict__ ind,
                                                         const float* __restrict__ zsum,
                                                         float* __restrict__ zm, int nqb, int nkb,
                                                         int ld) {
   __shared__ int lst[256];
-  const int row = blockIdx.x, tid = threadIdx.x;
+  __shared__ float4 part[4][32];
+  const int row = blockIdx.x, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int bh = row / nqb;
   uint4* p = reinterpret_cast<uint4*>(ind + i64(row) * ld);
   for (int x = tid; x < ld / 8; x += blockDim.x) p[x] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   const int cnt = min(max(rows.marg_cnt[row], 0), nkb);
   const int32_t* idx = rows.marg_idx + i64(row) * nkb;
-  float acc = 0.f;
+  const float4* z4 = reinterpret_cast<const float4*>(zsum + i64(bh) * nkb * kD) + lane;
+  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
   for (int b0 = 0; b0 < cnt; b0 += 256) {
     const int n = min(256, cnt - b0);
     __syncthreads();
@@ -171,13 +176,28 @@ __global__ void __launch_bounds__(128) indicator_kernel(sla_block_lists rows,
       if (jj >= 0 && jj < nkb) ind[i64(row) * ld + jj] = 0x3F80u;  // bf16 1.0
     }
     __syncthreads();
-#pragma unroll 8
-    for (int e = 0; e < n; ++e) {
-      const int jj = lst[e];
-      if (jj >= 0) acc += zsum[(i64(bh) * nkb + jj) * kD + tid];
+    int e = warp;
+    for (; e + 4 < n; e += 8) {  // two entries per step, independent chains
+      const int j0 = lst[e], j1 = lst[e + 4];
+      if (j0 >= 0) {
+        const float4 v = z4[i64(j0) * (kD / 4)];
+        acc0.x += v.x; acc0.y += v.y; acc0.z += v.z; acc0.w += v.w;
+      }
+      if (j1 >= 0) {
+        const float4 v = z4[i64(j1) * (kD / 4)];
+        acc1.x += v.x; acc1.y += v.y; acc1.z += v.z; acc1.w += v.w;
+      }
+    }
+    if (e < n && lst[e] >= 0) {
+      const float4 v = z4[i64(lst[e]) * (kD / 4)];
+      acc0.x += v.x; acc0.y += v.y; acc0.z += v.z; acc0.w += v.w;
     }
   }
-  zm[i64(row) * kD + tid] = acc;
+  part[warp][lane] = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+  __syncthreads();
+  // channel tid = 4 * lane' + c of part[w][lane']
+  const float* pf = reinterpret_cast<const float*>(&part[0][0]);
+  zm[i64(row) * kD + tid] = ((pf[tid] + pf[128 + tid]) + pf[256 + tid]) + pf[384 + tid];
 }
 
 // 2b. Gather GEMM: HM[bh] (Nqb x 16384) = Ind[bh] (Nqb x ld) @ H[bh] (ld x 16384).
