@@ -207,7 +207,8 @@ __device__ void compact_row(const int8_t* lab, int n, int32_t* idx_c,
 
 // ---------------------------------------------------------------------------
 // Classifier: one CTA per (bh, query block) row (64 threads for rows of up to
-// 1024 blocks, 256 above).
+// 1024 blocks, 256 above); top-k rows of up to 1024 blocks take the one-warp
+// variant below (classify_topk_warp_kernel), which makes the same cuts.
 //   1. P = softmax of the row's logits (fp32, fixed reduction order), kept as
 //      32-bit patterns: scores are non-negative, so the patterns order like
 //      the values;
@@ -569,6 +570,149 @@ __global__ void __launch_bounds__(CT) classify_kernel(const float* __restrict__ 
               a.rows.marg_idx + off, a.rows.marg_cnt + row, redi);
 }
 
+// Top-k classifier with one warp per row (rows of up to 32 * VPL blocks):
+// the same cuts as classify_kernel with no block-wide barrier.  Lane l holds
+// blocks j = l + 32 i (i < VPL) in registers.  The score at rank k is built
+// bit by bit from the top (largest pattern t with at least k + 1 scores >= t;
+// the count is a warp reduction); equal scores fill the remaining slots in
+// index order, and the lists come out of ballots in index order.
+template <int VPL>
+__global__ void __launch_bounds__(256) classify_topk_warp_kernel(const float* __restrict__ logits,
+                                                                   ClassifyArgs a, int nrows) {
+  const int row = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (row >= nrows) return;  // whole warps only; no block-wide barrier below
+  const unsigned full = 0xffffffffu;
+  const int nkb = a.nkb;
+  const float* lr = logits + i64(row) * nkb;
+  uint32_t pb[VPL];
+  // 1. softmax over the row (fixed order: lane-local in i, then a butterfly)
+  float x[VPL];
+  float m = -FLT_MAX;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    x[i] = j < nkb ? lr[j] : -FLT_MAX;
+    m = fmaxf(m, x[i]);
+  }
+  float inv = 1.f;
+  if (!a.from_prob) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(full, m, o));
+    float se = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (lane + 32 * i < nkb) se += expf(x[i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(full, se, o);
+    inv = 1.0f / se;
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    const float p = a.from_prob ? fmaxf(x[i], 0.f) : expf(x[i] - m) * inv;
+    if (a.scores && j < nkb) a.scores[i64(row) * nkb + j] = p;
+    pb[i] = j < nkb ? __float_as_uint(p) : 0u;
+  }
+  auto valid = [&](int i) { return lane + 32 * i < nkb; };
+  auto count_ge = [&](uint32_t t) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) c += (valid(i) && pb[i] >= t) ? 1u : 0u;
+    return __reduce_add_sync(full, c);
+  };
+  auto count_eq = [&](uint32_t t) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) c += (valid(i) && pb[i] == t) ? 1u : 0u;
+    return static_cast<int>(__reduce_add_sync(full, c));
+  };
+  // largest pattern strictly below t (0 if none)
+  auto max_below = [&](uint32_t t) {
+    uint32_t mb = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (valid(i) && pb[i] < t && pb[i] > mb) mb = pb[i];
+    return __reduce_max_sync(full, mb);
+  };
+  // pattern at rank k (0-based from the top) and the count strictly above it
+  auto select_rank = [&](int k, uint32_t& v, int& above) {
+    uint32_t t = 0;
+    for (int bit = 30; bit >= 0; --bit) {  // scores are >= 0: bit 31 is clear
+      const uint32_t c = t | (1u << bit);
+      if (count_ge(c) >= static_cast<uint32_t>(k + 1)) t = c;
+    }
+    v = t;
+    above = t == 0xFFFFFFFFu ? 0 : static_cast<int>(count_ge(t + 1));
+  };
+  // labels as bit masks over the slots: bit i of crit / kept = block
+  // lane + 32 i is critical / critical or marginal
+  static_assert(VPL <= 64, "slot masks hold 64 slots");
+  uint64_t crit = 0, kept = 0;
+  // blocks above v, and the first `fill` blocks equal to v in index order
+  auto label_top = [&](uint32_t v, int fill, uint64_t& bits) {
+    int base = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const bool eq = valid(i) && pb[i] == v;
+      const unsigned be = __ballot_sync(full, eq);
+      const int rank_eq = base + __popc(be & ((1u << lane) - 1u));
+      if (valid(i) && (pb[i] > v || (eq && rank_eq < fill))) bits |= 1ull << i;
+      base += __popc(be);
+    }
+  };
+  bool tie = false;
+  const int c = a.n_c;
+  if (c > 0) {
+    uint32_t v;
+    int above;
+    select_rank(c - 1, v, above);
+    label_top(v, c - above, crit);
+    if (a.tie_count && c < nkb) {  // gap between ranks c-1 and c
+      const uint32_t nxt = max_below(v);
+      const int eqcount = count_eq(v);
+      const float hi = __uint_as_float(v);
+      const float lo = (above + eqcount > c) ? hi : __uint_as_float(nxt);
+      tie |= (hi - lo) <= kTieEps * hi;
+    }
+  }
+  const int nm = min(a.n_m, nkb - c);
+  if (nm > 0) {
+    uint32_t v;
+    int above;
+    select_rank(c + nm - 1, v, above);
+    label_top(v, c + nm - above, kept);
+    if (a.tie_count && c + nm < nkb) {
+      const uint32_t nxt = max_below(v);
+      const int eqcount = count_eq(v);
+      const float hi = __uint_as_float(v);
+      const float lo = (above + eqcount > c + nm) ? hi : __uint_as_float(nxt);
+      tie |= (hi - lo) <= kTieEps * hi;
+    }
+  }
+  if (a.tie_count && lane == 0 && tie) atomicAdd(a.tie_count, 1);
+  // 3. mask row and the ascending lists
+  const i64 off = i64(row) * nkb;
+  int nc = 0, nmg = 0;
+  kept |= crit;  // (the marginal cut ranks below the critical one)
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    const bool is_c = (crit >> i) & 1ull, is_m = !is_c && ((kept >> i) & 1ull);
+    if (valid(i)) a.mask[off + j] = static_cast<int8_t>(is_c ? 2 : (is_m ? 1 : 0));
+    const unsigned bc = __ballot_sync(full, is_c);
+    const unsigned bm = __ballot_sync(full, is_m);
+    const unsigned lt = (1u << lane) - 1u;
+    if (is_c) a.rows.crit_idx[off + nc + __popc(bc & lt)] = j;
+    if (is_m) a.rows.marg_idx[off + nmg + __popc(bm & lt)] = j;
+    nc += __popc(bc);
+    nmg += __popc(bm);
+  }
+  if (lane == 0) {
+    a.rows.crit_cnt[row] = nc;
+    a.rows.marg_cnt[row] = nmg;
+  }
+}
+
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
                             const sla_block_lists& rows, float* scores,
                             int32_t* tie_count, cudaStream_t s, bool from_prob) {
@@ -589,9 +733,16 @@ cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
     e = cudaMemsetAsync(tie_count, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
   }
-  // short rows: small CTAs (cheap barriers, many rows per SM); long rows:
-  // more threads per row
-  if (g.nkb <= 1024) {
+  // top-k rows of up to 1024 blocks: one warp per row (measured faster than
+  // the CTA kernel there, slower for rows of 1920 blocks); otherwise small
+  // CTAs for short rows (cheap barriers, many rows per SM), more threads per
+  // row for long ones
+  const int nrows = g.BH * g.nqb;
+  if (g.mode == SLA_MASK_TOPK && g.nkb <= 1024) {
+    const int grid = (nrows + 7) / 8;
+    if (g.nkb <= 512) classify_topk_warp_kernel<16><<<grid, 256, 0, s>>>(logits, a, nrows);
+    else classify_topk_warp_kernel<32><<<grid, 256, 0, s>>>(logits, a, nrows);
+  } else if (g.nkb <= 1024) {
     if ((e = cudaFuncSetAttribute(classify_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(smem))) != cudaSuccess)
       return e;
