@@ -282,9 +282,10 @@ def run_ours(args, rank, world, local_rank):
             gk.data_ptr(), gv.data_ptr(), gw.data_ptr(), ws_b.data_ptr(), ws_b.numel(), sp))
 
     fused = sla.sla_forward_uses_tensor_cores(p) == 1 and (wl.frac_marg == 0 or wl.d == 128)
-    # kernels per step: pool x2, logits, classify | plan (+ W to bf16, summaries,
-    # indicator, gather GEMM) | fused attention (or attention + combine)
-    launches_per_step = 4 + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
+    # kernels per step: pool (Q and K in one launch), logits, classify | plan
+    # (+ W to bf16, summaries, indicator, gather GEMM) | fused attention (or
+    # attention + combine)
+    launches_per_step = 3 + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
         + (1 if (not fused and wl.frac_marg > 0) else 0) + (1 if fused else 2)
     if bwd:
         lin = wl.frac_marg > 0

@@ -36,8 +36,9 @@ bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box);
 
 // mask path
-cudaError_t launch_pool(const void* x, int dtype, float* out, int BH, int N,
-                        int d, int block, cudaStream_t s);
+// block means of Q (blocks of bq tokens) and K (blocks of bk) in one launch
+cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar, int BH,
+                        int N, int d, int bq, int bk, cudaStream_t s);
 cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
                           const Geom& g, cudaStream_t s);
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,

@@ -18,12 +18,21 @@ namespace sla {
 // reduction order (per-thread running sums, then a fixed tree in shared
 // memory), so the result is deterministic.
 
+// Block means of Q (blockIdx.z = 0, blocks of bq tokens) and K (z = 1,
+// blocks of bk) in one launch: one CTA per (block, bh); each thread sums a
+// 16-byte slice of every lanes-th token, then the slices' partial sums are
+// added in a fixed order.
 template <typename T>
-__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ x,
-                                                   float* __restrict__ out,
-                                                   int N, int d, int block) {
+__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, const T* __restrict__ xk,
+                                                   float* __restrict__ outq, float* __restrict__ outk,
+                                                   int N, int d, int bq, int bk) {
   constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
-  const int b = blockIdx.x, bh = blockIdx.y, nb = gridDim.x;
+  const bool isk = blockIdx.z == 1;
+  const int block = isk ? bk : bq, nb = (N + block - 1) / block;
+  const int b = blockIdx.x, bh = blockIdx.y;
+  if (b >= nb) return;
+  const T* x = isk ? xk : xq;
+  float* out = isk ? outk : outq;
   const int t0 = b * block, t1 = min(t0 + block, N), cnt = t1 - t0;
   const T* base = x + (i64(bh) * N) * d;
   const int vpt = d / VEC;                 // vectors per token
@@ -34,10 +43,21 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ x,
   for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
   for (int t = t0 + tl; t < t1; t += lanes) {
     const T* p = base + i64(t) * d + v * VEC;
+    if constexpr (sizeof(T) == 2) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(p);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-    for (int e = 0; e < VEC; e += 4) {
-      float4 f = load4(p + e);
-      acc[e] += f.x; acc[e + 1] += f.y; acc[e + 2] += f.z; acc[e + 3] += f.w;
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+        acc[2 * q] += f.x;
+        acc[2 * q + 1] += f.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < VEC; e += 4) {
+        float4 f = load4(p + e);
+        acc[e] += f.x; acc[e + 1] += f.y; acc[e + 2] += f.z; acc[e + 3] += f.w;
+      }
     }
   }
   __shared__ float part[256 * 8];  // lanes * d <= 256 * VEC
@@ -52,15 +72,16 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ x,
   }
 }
 
-cudaError_t launch_pool(const void* x, int dtype, float* out, int BH, int N,
-                        int d, int block, cudaStream_t s) {
-  dim3 grid((N + block - 1) / block, BH);
+cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar, int BH,
+                        int N, int d, int bq, int bk, cudaStream_t s) {
+  dim3 grid((N + min(bq, bk) - 1) / min(bq, bk), BH, 2);
   if (dtype == SLA_BF16)
-    pool_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), out, N, d, block);
+    pool_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
+                                                    static_cast<const __nv_bfloat16*>(k), qbar, kbar,
+                                                    N, d, bq, bk);
   else
-    pool_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), out,
-                                            N, d, block);
+    pool_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                            qbar, kbar, N, d, bq, bk);
   return cudaGetLastError();
 }
 

@@ -209,8 +209,7 @@ sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
   float* qbar = at<float>(ws, w.qbar);
   float* kbar = at<float>(ws, w.kbar);
   float* logits = at<float>(ws, w.logits);
-  SLA_CUDA(sla::launch_pool(q, g.dtype, qbar, g.BH, g.N, g.d, g.bq, s));
-  SLA_CUDA(sla::launch_pool(k, g.dtype, kbar, g.BH, g.N, g.d, g.bk, s));
+  SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, g.BH, g.N, g.d, g.bq, g.bk, s));
   SLA_CUDA(sla::launch_logits(qbar, kbar, logits, g, s));
   SLA_CUDA(sla::launch_classify(logits, g, mask, *rows, scores, tie_count, s));
   if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
