@@ -800,31 +800,57 @@ cudaError_t launch_rows_from_mask(const int8_t* mask, const Geom& g,
   return cudaGetLastError();
 }
 
-// One thread per (bh, key block): walk the column top to bottom.  Threads of
-// a warp read adjacent bytes of each mask row.
-__global__ void cols_from_mask_kernel(const int8_t* __restrict__ mask, int BH,
-                                      int nqb, int nkb, sla_block_lists cols) {
-  const i64 t = i64(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= i64(BH) * nkb) return;
-  const int bh = static_cast<int>(t / nkb), j = static_cast<int>(t % nkb);
-  int nc = 0, nm = 0;
-  const int8_t* col = mask + i64(bh) * nqb * nkb + j;
-  int32_t* ic = cols.crit_idx + t * nqb;
-  int32_t* im = cols.marg_idx + t * nqb;
-  for (int i = 0; i < nqb; ++i) {
-    const int8_t lb = col[i64(i) * nkb];
-    if (lb == 2) ic[nc++] = i;
-    else if (lb == 1) im[nm++] = i;
+// One CTA per (bh, 32 consecutive key blocks): 32-row slabs of those 32
+// mask columns go through shared memory (rows padded to 36 bytes, so the
+// column reads below hit 32 distinct banks); warp w then appends, for its
+// four columns, the slab's critical and marginal rows with two ballots each
+// -- lists stay ascending.
+__global__ void __launch_bounds__(256) cols_from_mask_kernel(const int8_t* __restrict__ mask, int BH,
+                                                            int nqb, int nkb, sla_block_lists cols) {
+  __shared__ int8_t tile[32][36];
+  const int bh = blockIdx.y, j0 = blockIdx.x * 32;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int8_t* mrow = mask + i64(bh) * nqb * nkb;
+  const int lr = tid / 8, lb = (tid % 8) * 4;  // loader: slab row, first of four columns
+  int nc[4] = {0, 0, 0, 0}, nm[4] = {0, 0, 0, 0};
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = 0; i0 < nqb; i0 += 32) {
+    __syncthreads();
+    const int i = i0 + lr;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + lb + q;
+      tile[lr][lb + q] = (i < nqb && j < nkb) ? mrow[i64(i) * nkb + j] : int8_t(0);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = warp + 8 * k, j = j0 + c;
+      if (j >= nkb) continue;  // warp-uniform
+      const int8_t v = tile[lane][c];
+      const unsigned bc = __ballot_sync(0xffffffffu, v == 2);
+      const unsigned bm = __ballot_sync(0xffffffffu, v == 1);
+      const i64 t = i64(bh) * nkb + j;
+      if (v == 2) cols.crit_idx[t * nqb + nc[k] + __popc(bc & lt)] = i0 + lane;
+      if (v == 1) cols.marg_idx[t * nqb + nm[k] + __popc(bm & lt)] = i0 + lane;
+      nc[k] += __popc(bc);
+      nm[k] += __popc(bm);
+    }
   }
-  cols.crit_cnt[t] = nc;
-  cols.marg_cnt[t] = nm;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int j = j0 + warp + 8 * k;
+    if (lane == 0 && j < nkb) {
+      cols.crit_cnt[i64(bh) * nkb + j] = nc[k];
+      cols.marg_cnt[i64(bh) * nkb + j] = nm[k];
+    }
+  }
 }
 
 cudaError_t launch_cols_from_mask(const int8_t* mask, const Geom& g,
                                   const sla_block_lists& cols, cudaStream_t s) {
-  const i64 n = i64(g.BH) * g.nkb;
-  cols_from_mask_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, s>>>(
-      mask, g.BH, g.nqb, g.nkb, cols);
+  dim3 grid((g.nkb + 31) / 32, g.BH);
+  cols_from_mask_kernel<<<grid, 256, 0, s>>>(mask, g.BH, g.nqb, g.nkb, cols);
   return cudaGetLastError();
 }
 
