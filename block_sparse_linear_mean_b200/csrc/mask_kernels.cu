@@ -9,6 +9,7 @@
 #include <float.h>
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace sla {
 
@@ -125,10 +126,18 @@ __global__ void __launch_bounds__(64) logits_kernel(const float* __restrict__ qb
       const float4 b1 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8 + 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      // paired fp32 FMAs: the same a * b + acc per entry, two entries per
+      // instruction
 #pragma unroll
-      for (int m = 0; m < 8; ++m)
+      for (int m = 0; m < 8; ++m) {
+        const float2 am = make_float2(a[m], a[m]);
 #pragma unroll
-        for (int n = 0; n < 8; ++n) acc[m][n] = fmaf(a[m], b[n], acc[m][n]);
+        for (int n = 0; n < 8; n += 2) {
+          const float2 r2 = fma2(am, make_float2(b[n], b[n + 1]), make_float2(acc[m][n], acc[m][n + 1]));
+          acc[m][n] = r2.x;
+          acc[m][n + 1] = r2.y;
+        }
+      }
     }
     __syncthreads();
   }
