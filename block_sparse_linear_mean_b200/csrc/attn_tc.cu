@@ -141,7 +141,8 @@ template <int D, int BQ, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmHM,
-               const __grid_constant__ CUtensorMap tmW, const int32_t* __restrict__ plan_cnt,
+               const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmOut,
+               const int32_t* __restrict__ plan_cnt,
                const uint32_t* __restrict__ plan_tiles, int plan_stride, AttnEpilogue ep,
                int32_t* status, int N, int nqt, float scale_log2, long long timeout_cycles,
                int debug_skip) {
@@ -745,13 +746,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] += lo[i];
         }
-        if (row < N) {
+        // bf16 into the staging tile (K stage 0, free: its last readers,
+        // the S and linear-branch MMAs, are done), in the 128-byte swizzled
+        // layout of the output's tensor map; rows past N are dropped by the
+        // store
+        const int ch = h * DH + c;  // first channel of these 32
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(ep.out + orow + c + 8 * q4) =
-                make_uint4(pack_bf16x2(o[8 * q4], o[8 * q4 + 1]), pack_bf16x2(o[8 * q4 + 2], o[8 * q4 + 3]),
-                           pack_bf16x2(o[8 * q4 + 4], o[8 * q4 + 5]), pack_bf16x2(o[8 * q4 + 6], o[8 * q4 + 7]));
-        }
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<uint4*>(base + offK + (ch / 64) * 16384 + sw128(r, (ch % 64) / 8 + q4)) =
+              make_uint4(pack_bf16x2(o[8 * q4], o[8 * q4 + 1]), pack_bf16x2(o[8 * q4 + 2], o[8 * q4 + 3]),
+                         pack_bf16x2(o[8 * q4 + 4], o[8 * q4 + 5]), pack_bf16x2(o[8 * q4 + 6], o[8 * q4 + 7]));
+      }
+    }
+    if (ep.out) {
+      // one TMA store per 64-channel chunk once all 256 threads have written
+      fence_async_smem();
+      asm volatile("bar.sync 2, 256;" ::: "memory");  // the softmax warps only
+      if (threadIdx.x == 64) {
+#pragma unroll
+        for (int c = 0; c < DC; ++c) tma_store_3d(&tmOut, sb + offK + c * 16384, c * 64, qt * kTileM, bh);
+        tma_store_commit();
+        tma_store_wait_read();  // the staging tile is read before the CTA ends
       }
     }
     if (row < N && h == 0)
@@ -785,7 +800,7 @@ bool make_map(CUtensorMap* m, const void* ptr, const Geom& g, int rows) {
 
 template <int D, int BQ, int BK>
 cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mhm, const CUtensorMap& mw, const int32_t* cnt,
+                     const CUtensorMap& mhm, const CUtensorMap& mw, const CUtensorMap& mo, const int32_t* cnt,
                      const uint32_t* tiles, const Geom& g, int nqt, const AttnEpilogue& ep,
                      int32_t* status, cudaStream_t s) {
   auto kern = attn_tc_kernel<D, BQ, BK>;
@@ -795,7 +810,7 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   const float scale_log2 = g.scale * 1.4426950408889634f;
   const bool debug = (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0;
   const long long timeout = debug ? (1ll << 24) : (1ll << 31);
-  kern<<<g.BH * nqt, kThreads, kSmemRequest, s>>>(mq, mk, mv, mhm, mw, cnt, tiles, g.nkb, ep, status,
+  kern<<<g.BH * nqt, kThreads, kSmemRequest, s>>>(mq, mk, mv, mhm, mw, mo, cnt, tiles, g.nkb, ep, status,
                                                   g.N, nqt, scale_log2, timeout, debug ? 1 : 0);
   return cudaGetLastError();
 }
@@ -853,9 +868,11 @@ cudaError_t launch_attn_tc_fused(const void* q, const void* k, const void* v, co
                                  int32_t* status, cudaStream_t s) {
   const int nqt = (g.N + kTileM - 1) / kTileM;
   const PlanPtrs pp = plan_ptrs(g, scratch);
-  CUtensorMap mq, mk, mv, mhm, mw;
+  CUtensorMap mq, mk, mv, mhm, mw, mo;
   if (!make_map(&mq, q, g, kTileM) || !make_map(&mk, k, g, g.bk) || !make_map(&mv, v, g, g.bk))
     return cudaErrorInvalidValue;
+  mo = mq;  // unused without a bf16 output
+  if (o.out && !make_map(&mo, o.out, g, kTileM)) return cudaErrorInvalidValue;
   AttnEpilogue ep;
   ep.o_s = o.o_s;
   ep.lse = o.lse;
@@ -878,7 +895,7 @@ cudaError_t launch_attn_tc_fused(const void* q, const void* k, const void* v, co
   }
 #define SLA_TC_CASE(D_, BQ_, BK_)                                                                 \
   if (g.d == D_ && g.bq == BQ_ && g.bk == BK_)                                                    \
-    return launch_t<D_, BQ_, BK_>(mq, mk, mv, mhm, mw, pp.cnt, pp.tiles, g, nqt, ep, status, s);
+    return launch_t<D_, BQ_, BK_>(mq, mk, mv, mhm, mw, mo, pp.cnt, pp.tiles, g, nqt, ep, status, s);
   SLA_TC_CASE(128, 64, 64)
   SLA_TC_CASE(128, 64, 128)
   SLA_TC_CASE(128, 128, 64)
