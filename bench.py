@@ -50,7 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the current kernel version (dram__bytes_read.sum +
 # dram__bytes_write.sum; command and figures in profiles/); absent = null.
 TRAFFIC_PER_LAUNCH = {
-    ("sla_1p3b", "attn_tc"): 506_977_280 + 90_916_352,
+    ("sla_1p3b", "attn_tc"): 507_041_280 + 92_068_608,
 }
 
 
