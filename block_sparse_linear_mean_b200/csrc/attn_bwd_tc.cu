@@ -182,7 +182,8 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   const uint32_t b_dfr = smem_u32(&bars[kL0 + 7]);   // df read (8 warps)
   const uint32_t b_dh2 = smem_u32(&bars[kL0 + 8]);   // dH^M of the second block in TMEM
   const uint32_t b_dz = smem_u32(&bars[kL0 + 9]);    // dz^M halves exchanged (8 warps)
-  static_assert((kL0 + 10) * 8 <= 512, "barrier block");
+  const uint32_t b_qt = smem_u32(&bars[kL0 + 10]);   // Q and dO copied into TMEM (8 warps)
+  static_assert((kL0 + 11) * 8 <= 512, "barrier block");
   float* red = reinterpret_cast<float*>(base + offRed);
   float* dd = reinterpret_cast<float*>(base + offDd);
 
@@ -234,6 +235,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     mbar_init(b_dfr, 8);
     mbar_init(b_dh2, 1);
     mbar_init(b_dz, 8);
+    mbar_init(b_qt, 8);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -248,6 +250,11 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   auto tS = [&](int b) { return tmem + 64u * static_cast<uint32_t>(b); };
   auto tP = [&](int b) { return tmem + 128u + 64u * static_cast<uint32_t>(b); };
   const uint32_t tQ = tmem + 256;
+  // during the main loop Q and dO also sit in TMEM (bf16 pairs, row m in
+  // lane m) as the A operands of S = Q K^T and dP = dO V^T, so those
+  // products read only K and V from shared memory; the linear epilogue
+  // reuses these columns afterwards
+  const uint32_t tQa = tmem + 384, tdOa = tmem + 448;
   BwdShared sh{bars, abort_flag, status, timeout};
 
   if (warp == 0) {
@@ -309,16 +316,14 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         tc_fence_after();
         const uint64_t dK = sdesc_add(dKV, s * kStageBytes), dV = sdesc_add(dK, kHalfBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oa = (kk / 4) * 16384 + (kk % 4) * 32;
+        for (int kk = 0; kk < D / 16; ++kk) {  // 16 channels = 8 TMEM columns of Q
           const uint32_t ob = (kk / 4) * 8192 + (kk % 4) * 32;
-          tc_mma(tS(b), sdesc_add(dQd, oa), sdesc_add(dK, ob), idesc_s, kk > 0);
+          tc_mma_ts(tS(b), tQa + kk * 8, sdesc_add(dK, ob), idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oa = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t ob = (kk / 4) * 8192 + (kk % 4) * 32;
-          tc_mma(tP(b), sdesc_add(ddO, oa), sdesc_add(dV, ob), idesc_s, kk > 0);
+          tc_mma_ts(tP(b), tdOa + kk * 8, sdesc_add(dV, ob), idesc_s, kk > 0);
         }
         tc_commit(b_s(b));
         return true;
@@ -335,6 +340,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         tc_commit(b_empty(s));
         return true;
       };
+      if (ok) ok = bwait(sh, b_qt, 0);  // Q and dO in TMEM
       if (ok) ok = issue_sdp(0);
       for (int u = 0; ok && u < U; ++u) {
         if (u + 1 < U) ok = issue_sdp(u + 1);
@@ -418,6 +424,34 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const float2 nl2 = make_float2(-lse2, -lse2);
     const float2 nd2 = make_float2(-dl, -dl);
     bool ok = true;
+    if (U > 0) {
+      // Q and dO of row r, channels [h D/2, (h + 1) D/2), into TMEM as bf16
+      // pairs (even channel in the low half), from their swizzled tiles
+      ok = __all_sync(full, bwait(sh, b_q, 0));
+      if (ok) {
+        uint32_t pq[D / 4], pd[D / 4];
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+          const int ch = h * (D / 2) + 8 * i;
+          const uint32_t off = (ch / 64) * 16384 + sw128(r, (ch % 64) / 8);
+          const uint4 vq = *reinterpret_cast<const uint4*>(base + offQ + off);
+          const uint4 vd = *reinterpret_cast<const uint4*>(base + offdO + off);
+          pq[4 * i] = vq.x; pq[4 * i + 1] = vq.y; pq[4 * i + 2] = vq.z; pq[4 * i + 3] = vq.w;
+          pd[4 * i] = vd.x; pd[4 * i + 1] = vd.y; pd[4 * i + 2] = vd.z; pd[4 * i + 3] = vd.w;
+        }
+        if constexpr (D == 128) {
+          tmem_st32u(tQa + lane_off + 32 * h, pq);
+          tmem_st32u(tdOa + lane_off + 32 * h, pd);
+        } else {
+          tmem_st16u(tQa + lane_off + 16 * h, pq);
+          tmem_st16u(tdOa + lane_off + 16 * h, pd);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_qt);
+    }
     int u = 0;
     for (int t = 0; ok && t < T; ++t) {
       const uint32_t desc = ptiles[t];
