@@ -84,12 +84,20 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
       *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
-    {  // z_j[a] from the rounded phi(K) the MMA uses
+    {  // z_j[a] from the rounded phi(K) the MMA uses (four chains, added
+       // in a fixed order)
       const int a = tid;
       const uint8_t* ch = base + offK + (a >> 6) * kChunk;
-      float z = 0.f;
-      for (int u = 0; u < valid; ++u) z += bf16_at(ch, u, a & 63);
-      zsum[(i64(bh) * nkb + j) * kD + a] = z;
+      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+      int u = 0;
+      for (; u + 4 <= valid; u += 4) {
+        z0 += bf16_at(ch, u, a & 63);
+        z1 += bf16_at(ch, u + 1, a & 63);
+        z2 += bf16_at(ch, u + 2, a & 63);
+        z3 += bf16_at(ch, u + 3, a & 63);
+      }
+      for (; u < valid; ++u) z0 += bf16_at(ch, u, a & 63);
+      zsum[(i64(bh) * nkb + j) * kD + a] = (z0 + z1) + (z2 + z3);
     }
     fence_async_smem();
     tc_fence_before();
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
     tma_store_2d(&tmH, sb, 0, row0);
     tma_store_2d(&tmH, sb + 16384, 64, row0);
     tma_store_commit();
-    tma_store_wait_all();
+    tma_store_wait_read();  // the staging tile is read before the CTA ends
   }
   tc_fence_before();
   __syncthreads();
@@ -203,15 +211,15 @@ __global__ void __launch_bounds__(128) indicator_kernel(sla_block_lists rows,
 // 2b. Gather GEMM: HM[bh] (Nqb x 16384) = Ind[bh] (Nqb x ld) @ H[bh] (ld x 16384).
 //     Persistent: one CTA per SM walks output tiles of 128 x 256 (consecutive
 //     tiles share their H columns, so the CTAs working at one time read each
-//     H tile from L2 after the first).  K step 64, 3-stage TMA ring; warp 0
+//     H tile from L2 after the first).  K step 64, 4-stage TMA ring; warp 0
 //     loads, warp 1 issues tcgen05.mma (A K-major, B MN-major) into one of
-//     two TMEM accumulators, warps 2-5 drain the other into a swizzled bf16
-//     tile that TMA stores write out -- a tile's epilogue overlaps the next
-//     tile's products.
-constexpr int kGStages = 3;
+//     two TMEM accumulators, warps 2-5 drain the other, 128 columns at a
+//     time, into a swizzled bf16 half tile that TMA stores write out -- a
+//     tile's epilogue overlaps the next tile's products.
+constexpr int kGStages = 4;
 constexpr uint32_t kGA = 16384, kGB = 32768, kGStage = kGA + kGB;
-constexpr uint32_t kGStaging = kGStages * kGStage;       // 64 KB bf16 output tile
-constexpr uint32_t kGBars = kGStaging + 65536;
+constexpr uint32_t kGStaging = kGStages * kGStage;       // 32 KB bf16 half tile
+constexpr uint32_t kGBars = kGStaging + 32768;
 constexpr size_t kGSmem = kGBars + 256 + 1024;
 
 __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
@@ -294,34 +302,38 @@ __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
       int m0, n0, bh;
       coords(t, m0, n0, bh);
       ok = wait_bounded(b_acc_full(a), (it >> 1) & 1, status, kTimeout);
-      // the previous tile's stores have read the staging tile
-      if (threadIdx.x == 64) tma_store_wait_read();
-      ok = bar_sync_and(1, 128, ok);  // all four warps take the same branch
-      if (!ok) break;
       tc_fence_after();
+      for (int hf = 0; hf < 2; ++hf) {  // (every warp reaches the barrier below)
+        // the previous stores have read the staging half tile
+        if (threadIdx.x == 64) tma_store_wait_read();
+        ok = bar_sync_and(1, 128, ok);  // all four warps take the same branch
+        if (!ok) break;
 #pragma unroll
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        float v[32];
-        tmem_ld32(tmem + 256 * a + lane_off + c0, v);
-        tmem_wait_ld();
-        reg_fence<32>(v);
-        uint8_t* ch = base + kGStaging + (c0 >> 6) * 16384;  // 4 chunks of [128 rows][64 cols]
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem + 256 * a + 128 * hf + lane_off + c0, v);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          uint8_t* ch = base + kGStaging + (c0 >> 6) * 16384;  // 2 chunks of [128 rows][64 cols]
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(ch + sw128(r, ((c0 & 63) >> 3) + q)) =
-              make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                         pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-      }
-      // accumulator free for tile it + 2
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_acc_empty(a));
-      fence_async_smem();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (threadIdx.x == 64) {
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(ch + sw128(r, ((c0 & 63) >> 3) + q)) =
+                make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        }
+        if (hf == 1) {  // accumulator free for tile it + 2
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_acc_empty(a));
+        }
+        fence_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 64) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_store_3d(&tmC, sb + kGStaging + c * 16384, n0 + c * 64, m0, bh);
-        tma_store_commit();
+          for (int c = 0; c < 2; ++c)
+            tma_store_3d(&tmC, sb + kGStaging + c * 16384, n0 + 128 * hf + c * 64, m0, bh);
+          tma_store_commit();
+        }
       }
     }
     if (threadIdx.x == 64) tma_store_wait_all();
