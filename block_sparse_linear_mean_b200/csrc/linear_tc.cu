@@ -152,6 +152,140 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
   }
 }
 
+// Persistent summaries for key blocks of 64 tokens: each CTA walks the items
+// w = blockIdx.x, blockIdx.x + gridDim.x, ... (item w = key block w % nkb of
+// head w / nkb) with two K/V buffers, so the next item's tiles load while
+// the current one is processed; after its products a buffer is the staging
+// tile of that item's H, and the next load into it waits until the store
+// has read it.  Same steps as lin_summary_tc_kernel.
+__global__ void __launch_bounds__(128) lin_summary_persist_kernel(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const __grid_constant__ CUtensorMap tmH, float* __restrict__ zsum, int N, int nkb, int nitems,
+    int32_t* status) {
+  constexpr int BK = 64;
+  constexpr uint32_t kChunk = BK * 128;  // bytes of one 64-column chunk
+  constexpr uint32_t kBuf = 4 * kChunk;  // K (2 chunks) then V (2 chunks); 32 KB = one H tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  const uint32_t sb = smem_u32(base);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 2 * kBuf);
+  auto b_tma = [&](int b) { return smem_u32(&bars[b]); };
+  const uint32_t b_mma = smem_u32(&bars[2]);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(&bars[3]);
+  const int tid = threadIdx.x, warp = tid / 32;
+  if (tid == 0) {
+    mbar_init(b_tma(0), 1);
+    mbar_init(b_tma(1), 1);
+    mbar_init(b_mma, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tslot), 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  auto issue_load = [&](int w, int b) {  // (one thread)
+    const int j = w % nkb, bh = w / nkb;
+    const uint32_t dst = sb + b * kBuf;
+    mbar_expect_tx(b_tma(b), kBuf);
+    for (int c = 0; c < 2; ++c) {
+      tma_load_3d(dst + c * kChunk, &tmK, c * 64, j * BK, bh, b_tma(b));
+      tma_load_3d(dst + 2 * kChunk + c * kChunk, &tmV, c * 64, j * BK, bh, b_tma(b));
+    }
+  };
+  if (tid == 0 && static_cast<int>(blockIdx.x) < nitems) issue_load(blockIdx.x, 0);
+  bool ok = true;
+  int k = 0;
+  for (int w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++k) {
+    const int b = k & 1, j = w % nkb, bh = w / nkb;
+    const int valid = min(BK, N - j * BK);
+    uint8_t* buf = base + b * kBuf;
+    const uint32_t sbuf = sb + b * kBuf;
+    // next item into the other buffer, once the previous item's H store has
+    // read it
+    if (tid == 0 && w + static_cast<int>(gridDim.x) < nitems) {
+      tma_store_wait_read();
+      issue_load(w + gridDim.x, b ^ 1);
+    }
+    ok = __syncthreads_and(wait_bounded(b_tma(b), (k >> 1) & 1, status, kTimeout));
+    if (!ok) break;
+    for (int x = tid; x < BK * 16; x += 128) {
+      const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
+      uint4* p = reinterpret_cast<uint4*>(buf + chunk * kChunk + sw128(row, u));
+      *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+    {  // z_j[a] from the rounded phi(K) the MMA uses (four chains, added
+       // in a fixed order)
+      const int a = tid;
+      const uint8_t* ch = buf + (a >> 6) * kChunk;
+      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+      int u = 0;
+      for (; u + 4 <= valid; u += 4) {
+        z0 += bf16_at(ch, u, a & 63);
+        z1 += bf16_at(ch, u + 1, a & 63);
+        z2 += bf16_at(ch, u + 2, a & 63);
+        z3 += bf16_at(ch, u + 3, a & 63);
+      }
+      for (; u < valid; ++u) z0 += bf16_at(ch, u, a & 63);
+      zsum[(i64(bh) * nkb + j) * kD + a] = (z0 + z1) + (z2 + z3);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+        tc_mma(tmem, sdesc(sbuf + kk * 2048, kChunk, 1024), sdesc(sbuf + 2 * kChunk + kk * 2048, kChunk, 1024),
+               idesc, kk > 0);
+      tc_commit(b_mma);
+    }
+    ok = __syncthreads_and(wait_bounded(b_mma, k & 1, status, kTimeout));
+    if (!ok) break;
+    // TMEM lane a -> bf16 row a of a 128B-swizzled staging tile (this buffer)
+    tc_fence_after();
+    {
+      const int a = tid;
+      const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + c0, v);
+        tmem_wait_ld();
+        reg_fence<32>(v);
+        uint8_t* ch = buf + (c0 >> 6) * 16384;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(ch + sw128(a, ((c0 & 63) >> 3) + q)) =
+              make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // (also: every TMEM read done before the next item's products)
+    if (tid == 0) {
+      const int row0 = (bh * nkb + j) * kD;
+      tma_store_2d(&tmH, sbuf, 0, row0);
+      tma_store_2d(&tmH, sbuf + 16384, 64, row0);
+      tma_store_commit();
+    }
+  }
+  if (tid == 0) tma_store_wait_all();
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  if (!ok) {  // let in-flight copies drain (bounded)
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000) __nanosleep(1000);
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // 2a. Marginal indicator Ind[bh, i, j] (bf16 0/1, row stride ld) from the
 //     CSR marginal lists, and z^M_i = sum of z_j over the list (fp32): one
@@ -676,8 +810,13 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
     const size_t smem = std::max<size_t>(4 * size_t(g.bk) * 128 + 64 + 1024, 48 * 1024);
     dim3 grid(g.nkb, g.BH);
     if (g.bk == 64) {
-      if ((e = set_smem(lin_summary_tc_kernel<64>, smem)) != cudaSuccess) return e;
-      lin_summary_tc_kernel<64><<<grid, 128, smem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, status);
+      // persistent: three CTAs per SM (two 32 KB buffers each; 3 x 128 TMEM
+      // columns)
+      const size_t psmem = 2 * 32768 + 256 + 1024;
+      if ((e = set_smem(lin_summary_persist_kernel, psmem)) != cudaSuccess) return e;
+      const int nitems = g.BH * g.nkb;
+      const int pgrid = std::min(nitems, 3 * sm_count());
+      lin_summary_persist_kernel<<<pgrid, 128, psmem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, nitems, status);
     } else {
       if ((e = set_smem(lin_summary_tc_kernel<128>, smem)) != cudaSuccess) return e;
       lin_summary_tc_kernel<128><<<grid, 128, smem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, status);
