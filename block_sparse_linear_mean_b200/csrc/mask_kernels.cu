@@ -21,13 +21,15 @@ namespace sla {
 
 // Block means of Q (blockIdx.z = 0, blocks of bq tokens) and K (z = 1,
 // blocks of bk) in one launch: one CTA per (block, bh); each thread sums a
-// 16-byte slice of every lanes-th token, then the slices' partial sums are
-// added in a fixed order.
+// 16-byte slice of every lanes-th token (the loads of kU such tokens are
+// issued together, then added in token order), then the slices' partial
+// sums are added in a fixed order.
 template <typename T>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, const T* __restrict__ xk,
                                                    float* __restrict__ outq, float* __restrict__ outk,
                                                    int N, int d, int bq, int bk) {
   constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
+  constexpr int kU = 4;                // loads in flight per thread
   const bool isk = blockIdx.z == 1;
   const int block = isk ? bk : bq, nb = (N + block - 1) / block;
   const int b = blockIdx.x, bh = blockIdx.y;
@@ -42,22 +44,28 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, con
   float acc[VEC];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-  for (int t = t0 + tl; t < t1; t += lanes) {
-    const T* p = base + i64(t) * d + v * VEC;
-    if constexpr (sizeof(T) == 2) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(p);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  for (int t = t0 + tl; t < t1; t += kU * lanes) {
+    uint4 raw[kU];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
-        acc[2 * q] += f.x;
-        acc[2 * q + 1] += f.y;
-      }
-    } else {
+    for (int u = 0; u < kU; ++u) {
+      const int tt = t + u * lanes;
+      raw[u] = tt < t1 ? __ldg(reinterpret_cast<const uint4*>(base + i64(tt) * d + v * VEC))
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-      for (int e = 0; e < VEC; e += 4) {
-        float4 f = load4(p + e);
-        acc[e] += f.x; acc[e + 1] += f.y; acc[e + 2] += f.z; acc[e + 3] += f.w;
+    for (int u = 0; u < kU; ++u) {
+      if (t + u * lanes >= t1) break;
+      const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] += __uint_as_float(w[q]);
       }
     }
   }
@@ -644,12 +652,6 @@ __global__ void __launch_bounds__(256) classify_topk_warp_kernel(const float* __
     pb[i] = j < nkb ? __float_as_uint(p) : 0u;
   }
   auto valid = [&](int i) { return lane + 32 * i < nkb; };
-  auto count_ge = [&](uint32_t t) {
-    uint32_t c = 0;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) c += (valid(i) && pb[i] >= t) ? 1u : 0u;
-    return __reduce_add_sync(full, c);
-  };
   auto count_eq = [&](uint32_t t) {
     uint32_t c = 0;
 #pragma unroll
@@ -664,15 +666,35 @@ __global__ void __launch_bounds__(256) classify_topk_warp_kernel(const float* __
       if (valid(i) && pb[i] < t && pb[i] > mb) mb = pb[i];
     return __reduce_max_sync(full, mb);
   };
-  // pattern at rank k (0-based from the top) and the count strictly above it
-  auto select_rank = [&](int k, uint32_t& v, int& above) {
-    uint32_t t = 0;
+  // patterns at ranks k1 and k2 (0-based from the top), searched side by
+  // side so the two chains of warp reductions overlap, and the counts
+  // strictly above them (the thresholds are >= 1 and the empty slots hold
+  // 0, so empty slots never count)
+  auto select_rank2 = [&](int k1, int k2, uint32_t& v1, int& above1, uint32_t& v2, int& above2) {
+    uint32_t t1 = 0, t2 = 0;
     for (int bit = 30; bit >= 0; --bit) {  // scores are >= 0: bit 31 is clear
-      const uint32_t c = t | (1u << bit);
-      if (count_ge(c) >= static_cast<uint32_t>(k + 1)) t = c;
+      const uint32_t c1 = t1 | (1u << bit), c2 = t2 | (1u << bit);
+      uint32_t n1 = 0, n2 = 0;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        n1 += pb[i] >= c1 ? 1u : 0u;
+        n2 += pb[i] >= c2 ? 1u : 0u;
+      }
+      n1 = __reduce_add_sync(full, n1);
+      n2 = __reduce_add_sync(full, n2);
+      if (n1 >= static_cast<uint32_t>(k1 + 1)) t1 = c1;
+      if (n2 >= static_cast<uint32_t>(k2 + 1)) t2 = c2;
     }
-    v = t;
-    above = t == 0xFFFFFFFFu ? 0 : static_cast<int>(count_ge(t + 1));
+    v1 = t1;
+    v2 = t2;
+    uint32_t a1 = 0, a2 = 0;  // (t < 2^31, so t + 1 does not wrap)
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      a1 += pb[i] > t1 ? 1u : 0u;
+      a2 += pb[i] > t2 ? 1u : 0u;
+    }
+    above1 = static_cast<int>(__reduce_add_sync(full, a1));
+    above2 = static_cast<int>(__reduce_add_sync(full, a2));
   };
   // labels as bit masks over the slots: bit i of crit / kept = block
   // lane + 32 i is critical / critical or marginal
@@ -692,10 +714,15 @@ __global__ void __launch_bounds__(256) classify_topk_warp_kernel(const float* __
   };
   bool tie = false;
   const int c = a.n_c;
+  const int nm = min(a.n_m, nkb - c);
+  // the critical cut at rank c - 1, the marginal one at rank c + nm - 1
+  // (an absent cut repeats the other's search)
+  uint32_t v_c, v_m;
+  int above_c, above_m;
+  select_rank2(c > 0 ? c - 1 : c + nm - 1, nm > 0 ? c + nm - 1 : c - 1, v_c, above_c, v_m, above_m);
   if (c > 0) {
-    uint32_t v;
-    int above;
-    select_rank(c - 1, v, above);
+    const uint32_t v = v_c;
+    const int above = above_c;
     label_top(v, c - above, crit);
     if (a.tie_count && c < nkb) {  // gap between ranks c-1 and c
       const uint32_t nxt = max_below(v);
@@ -705,11 +732,9 @@ __global__ void __launch_bounds__(256) classify_topk_warp_kernel(const float* __
       tie |= (hi - lo) <= kTieEps * hi;
     }
   }
-  const int nm = min(a.n_m, nkb - c);
   if (nm > 0) {
-    uint32_t v;
-    int above;
-    select_rank(c + nm - 1, v, above);
+    const uint32_t v = v_m;
+    const int above = above_m;
     label_top(v, c + nm - above, kept);
     if (a.tie_count && c + nm < nkb) {
       const uint32_t nxt = max_below(v);
