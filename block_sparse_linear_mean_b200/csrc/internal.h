@@ -34,13 +34,20 @@ constexpr int kMaxBlocks = 8192;                     // Nqb, Nkb limit
 bool tma_available();
 bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box);
+bool encode_f32_map(void* map, const void* ptr, int rank, const uint64_t* dims,
+                    const uint64_t* strides, const uint32_t* box);
 
 // mask path
-// block means of Q (blocks of bq tokens) and K (blocks of bk) in one launch
-cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar, int BH,
-                        int N, int d, int bq, int bk, cudaStream_t s);
+// block means of Q (blocks of bq tokens) and K (blocks of bk) in one launch;
+// with qlo/klo given, split as hi (in qbar/kbar) + lo, both tf32
+cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar,
+                        float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s);
 cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
                           const Geom& g, cudaStream_t s);
+// the same logits on the tensor cores from the split means (logits_tc.cu)
+bool logits_tc_supported(const Geom& g);
+cudaError_t launch_logits_tc(const float* qhi, const float* qlo, const float* khi, const float* klo,
+                             float* logits, const Geom& g, int32_t* status, cudaStream_t s);
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
                             const sla_block_lists& rows, float* scores,
                             int32_t* tie_count, cudaStream_t s, bool from_prob = false);

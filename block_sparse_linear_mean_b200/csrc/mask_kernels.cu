@@ -23,10 +23,13 @@ namespace sla {
 // blocks of bk) in one launch: one CTA per (block, bh); each thread sums a
 // 16-byte slice of every lanes-th token (the loads of kU such tokens are
 // issued together, then added in token order), then the slices' partial
-// sums are added in a fixed order.
+// sums are added in a fixed order.  With lo arrays given, each mean m is
+// written split for the tf32 tensor-core logits: hi = tf32(m) in out and
+// lo = tf32(m - hi) in lo (m - hi is exact in fp32).
 template <typename T>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, const T* __restrict__ xk,
                                                    float* __restrict__ outq, float* __restrict__ outk,
+                                                   float* __restrict__ loq, float* __restrict__ lok,
                                                    int N, int d, int bq, int bk) {
   constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
   constexpr int kU = 4;                // loads in flight per thread
@@ -36,6 +39,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, con
   if (b >= nb) return;
   const T* x = isk ? xk : xq;
   float* out = isk ? outk : outq;
+  float* lo = isk ? lok : loq;
   const int t0 = b * block, t1 = min(t0 + block, N), cnt = t1 - t0;
   const T* base = x + (i64(bh) * N) * d;
   const int vpt = d / VEC;                 // vectors per token
@@ -77,20 +81,28 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, con
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float s = 0.f;
     for (int j = 0; j < lanes; ++j) s += part[j * d + c];
-    out[(i64(bh) * nb + b) * d + c] = s * inv;
+    const float m = s * inv;
+    const i64 o = (i64(bh) * nb + b) * d + c;
+    if (lo) {
+      const float hi = to_tf32(m);
+      out[o] = hi;
+      lo[o] = to_tf32(m - hi);
+    } else {
+      out[o] = m;
+    }
   }
 }
 
-cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar, int BH,
-                        int N, int d, int bq, int bk, cudaStream_t s) {
+cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar,
+                        float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s) {
   dim3 grid((N + min(bq, bk) - 1) / min(bq, bk), BH, 2);
   if (dtype == SLA_BF16)
     pool_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
                                                     static_cast<const __nv_bfloat16*>(k), qbar, kbar,
-                                                    N, d, bq, bk);
+                                                    qlo, klo, N, d, bq, bk);
   else
     pool_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                            qbar, kbar, N, d, bq, bk);
+                                            qbar, kbar, qlo, klo, N, d, bq, bk);
   return cudaGetLastError();
 }
 

@@ -70,7 +70,7 @@ bool has_linear_branch(const Geom& g) { return g.linear; }
 
 
 // Workspace layouts (each region 256-byte aligned).
-struct MaskWs { size_t qbar, kbar, logits, total; };
+struct MaskWs { size_t qbar, kbar, qlo, klo, logits, total; };
 struct FwdWs { size_t o_s, hsum, zsum, lintc, tc, total; };
 struct BwdWs { size_t delta, gbuf, hsum, zsum, dhm, dzm, dwp, plans, lin, total; };
 
@@ -87,6 +87,11 @@ MaskWs mask_ws(const Geom& g) {
   size_t off = kStatusBytes;
   w.qbar = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d);
   w.kbar = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+  w.qlo = w.klo = off;  // (the tf32 lo parts, for the tensor-core logits)
+  if (sla::logits_tc_supported(g)) {
+    w.qlo = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d);
+    w.klo = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
+  }
   w.logits = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.nkb);
   w.total = off;
   return w;
@@ -209,8 +214,16 @@ sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
   float* qbar = at<float>(ws, w.qbar);
   float* kbar = at<float>(ws, w.kbar);
   float* logits = at<float>(ws, w.logits);
-  SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, g.BH, g.N, g.d, g.bq, g.bk, s));
-  SLA_CUDA(sla::launch_logits(qbar, kbar, logits, g, s));
+  if (sla::logits_tc_supported(g)) {
+    float* qlo = at<float>(ws, w.qlo);
+    float* klo = at<float>(ws, w.klo);
+    SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, qlo, klo, g.BH, g.N, g.d, g.bq, g.bk, s));
+    SLA_CUDA(sla::launch_logits_tc(qbar, qlo, kbar, klo, logits, g, at<int32_t>(ws, 0), s));
+  } else {
+    SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, nullptr, nullptr, g.BH, g.N, g.d, g.bq, g.bk,
+                              s));
+    SLA_CUDA(sla::launch_logits(qbar, kbar, logits, g, s));
+  }
   SLA_CUDA(sla::launch_classify(logits, g, mask, *rows, scores, tie_count, s));
   if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
   return SLA_OK;

@@ -91,6 +91,19 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// kind::tf32: A and B are fp32 words in shared memory of which the tensor
+// core uses the tf32 part (sign, exponent, top 10 mantissa bits); fp32
+// accumulator.
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Same with the A operand in tensor memory (K-major; two 16-bit elements per
 // 32-bit column, row m in lane m).
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -288,6 +301,21 @@ constexpr uint32_t idesc_bf16(int m, int n, int a_mn, int b_mn) {
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+
+// Instruction descriptor of kind::tf32 (A and B format 2), fp32
+// accumulator, A and B K-major.
+constexpr uint32_t idesc_tf32(int m, int n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// fp32 -> tf32 (round to nearest, ties away from zero), as an fp32 word
+// with the low 13 mantissa bits cleared.
+__device__ __forceinline__ float to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r & 0xFFFFE000u);
+}
 
 // 2D tiled TMA load (x innermost, in elements).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,

@@ -21,21 +21,32 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool tma_available() { return encode_fn() != nullptr; }
 
-// bf16 tensor of rank 2 or 3 (dims[0] innermost, strides in bytes for dims
+// Tensor of rank 2 or 3 (dims[0] innermost, strides in bytes for dims
 // 1..rank-1), 128-byte swizzle, out-of-range elements read as zero.
-bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
-                     const uint64_t* strides, const uint32_t* box) {
+static bool encode_map(CUtensorMapDataType type, void* map, const void* ptr, int rank,
+                       const uint64_t* dims, const uint64_t* strides, const uint32_t* box) {
   auto fn = encode_fn();
   if (!fn || rank < 2 || rank > 3) return false;
   cuuint64_t d[3], st[2];
   cuuint32_t b[3], e[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i < rank - 1; ++i) st[i] = strides[i];
-  CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+  CUresult r = fn(static_cast<CUtensorMap*>(map), type, rank,
                   const_cast<void*>(ptr), d, st, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box) {
+  return encode_map(CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, map, ptr, rank, dims, strides, box);
+}
+
+// Same for an fp32 tensor.
+bool encode_f32_map(void* map, const void* ptr, int rank, const uint64_t* dims,
+                    const uint64_t* strides, const uint32_t* box) {
+  return encode_map(CU_TENSOR_MAP_DATA_TYPE_FLOAT32, map, ptr, rank, dims, strides, box);
 }
 
 }  // namespace sla

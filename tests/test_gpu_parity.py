@@ -49,8 +49,10 @@ def case(request):
 def test_mask_matches_oracle(case):
     name, wl, x, t, ref = case
     p = sla.params_from(t["q"], wl)
-    got = sla.build_mask(p, t["q"], t["k"], want_scores=True, want_cols=True)
+    ws = sla.workspace(p, sla.SLA_OP_MASK, "cuda")
+    got = sla.build_mask(p, t["q"], t["k"], want_scores=True, want_cols=True, ws=ws)
     torch.cuda.synchronize()
+    assert sla.check_device_status(ws) == sla.SLA_OK
     scores = to_np(got["scores"])
     np.testing.assert_allclose(scores, ref["scores"], rtol=2e-5, atol=1e-7)
     mask = got["mask"].cpu().numpy()
