@@ -73,10 +73,23 @@ __device__ __forceinline__ uint32_t entry(int blk, uint32_t flags) {
   return kPresent | (flags << 13) | static_cast<uint32_t>(blk);
 }
 
-__global__ void plan_kernel(sla_block_lists rows, int BH, int nqb, int nkb, int nqt, int bq,
-                            int bk, int32_t* __restrict__ cnt, uint32_t* __restrict__ tiles) {
-  const int tile = blockIdx.x * blockDim.x + threadIdx.x;
-  if (tile >= BH * nqt) return;
+// One warp per query tile: the tile's query blocks' critical lists are
+// scattered into per-warp bitmaps over the key blocks (membership a, b),
+// then read back in key order (a warp scan of the words' popcounts gives
+// each lane its output slot), so the union comes out ascending with its
+// membership flags whatever the lists' order; entries outside [0, nkb) are
+// skipped and repeated entries collapse.
+constexpr int kPlanWarps = 4;
+
+__global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(sla_block_lists rows, int BH, int nqb,
+                                                               int nkb, int nqt, int bq, int bk,
+                                                               int32_t* __restrict__ cnt,
+                                                               uint32_t* __restrict__ tiles) {
+  __shared__ uint32_t bits[kPlanWarps][2][kMaxBlocks / 32];
+  const unsigned full = 0xffffffffu;
+  const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tile = blockIdx.x * kPlanWarps + w;
+  if (tile >= BH * nqt) return;  // whole warps; no block-wide barrier below
   const int bh = tile / nqt, qt = tile % nqt;
   const int qa = bq == 128 ? qt : 2 * qt;
   const int qb = (bq == 64 && 2 * qt + 1 < nqb) ? 2 * qt + 1 : -1;
@@ -91,30 +104,51 @@ __global__ void plan_kernel(sla_block_lists rows, int BH, int nqb, int nkb, int 
     nb = min(max(rows.crit_cnt[rb], 0), nkb);
     lb = rows.crit_idx + i64(rb) * nkb;
   }
-  uint32_t* out = tiles + i64(tile) * nkb;
-  int ia = 0, ib = 0, nt = 0;
-  uint32_t pending = 0;
-  const int per_tile = kTileN / bk;  // 1 or 2 entries per key tile
-  int in_tile = 0;
-  while (ia < na || ib < nb) {
-    const int a = ia < na ? la[ia] : 0x7fffffff;
-    const int b = ib < nb ? lb[ib] : 0x7fffffff;
-    int blk;
-    uint32_t f;
-    if (a == b) { blk = a; f = fa | 2u; ++ia; ++ib; }
-    else if (a < b) { blk = a; f = fa; ++ia; }
-    else { blk = b; f = 2u; ++ib; }
-    if (blk < 0 || blk >= nkb) continue;  // malformed list entry
-    pending |= entry(blk, f) << (16 * in_tile);
-    if (++in_tile == per_tile) {
-      out[nt++] = pending;
-      pending = 0;
-      in_tile = 0;
-      if (nt == nkb) break;  // only reachable with duplicated list entries
-    }
+  const int nw = (nkb + 31) / 32;
+  uint32_t* ba = bits[w][0];
+  uint32_t* bb = bits[w][1];
+  for (int i = lane; i < nw; i += 32) { ba[i] = 0u; bb[i] = 0u; }
+  __syncwarp();
+  for (int e = lane; e < na; e += 32) {
+    const int blk = la[e];
+    if (blk >= 0 && blk < nkb) atomicOr(&ba[blk >> 5], 1u << (blk & 31));
   }
-  if (in_tile && nt < nkb) out[nt++] = pending;
-  cnt[tile] = nt;
+  for (int e = lane; e < nb; e += 32) {
+    const int blk = lb[e];
+    if (blk >= 0 && blk < nkb) atomicOr(&bb[blk >> 5], 1u << (blk & 31));
+  }
+  __syncwarp();
+  const int per_tile = kTileN / bk;  // 1 or 2 entries per key tile
+  uint32_t* out = tiles + i64(tile) * nkb;
+  uint16_t* out16 = reinterpret_cast<uint16_t*>(out);  // entry r of a packed pair list
+  int base = 0;
+  for (int w0 = 0; w0 < nw; w0 += 32) {
+    const int i = w0 + lane;
+    const uint32_t xa = i < nw ? ba[i] : 0u, xb = i < nw ? bb[i] : 0u;
+    uint32_t x = xa | xb;
+    const int c = __popc(x);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int r = base + incl - c;
+    while (x) {
+      const int bit = __ffs(x) - 1;
+      x &= x - 1u;
+      const uint32_t f = (((xa >> bit) & 1u) ? fa : 0u) | (((xb >> bit) & 1u) ? 2u : 0u);
+      const uint32_t en = entry(i * 32 + bit, f);
+      if (per_tile == 2) out16[r] = static_cast<uint16_t>(en);
+      else out[r] = en;
+      ++r;
+    }
+    base += __shfl_sync(full, incl, 31);
+  }
+  if (lane == 0) {
+    if (per_tile == 2 && (base & 1)) out16[base] = 0;  // empty second entry
+    cnt[tile] = (base + per_tile - 1) / per_tile;
+  }
 }
 
 // ------------------------------------------------------------------ kernel
@@ -848,7 +882,7 @@ cudaError_t launch_attn_plan(const Geom& g, const sla_block_lists& rows, void* s
   const int nqt = (g.N + kTileM - 1) / kTileM;
   const size_t ntiles = static_cast<size_t>(g.BH) * nqt;
   const PlanPtrs pp = plan_ptrs(g, scratch);
-  plan_kernel<<<static_cast<unsigned>((ntiles + 127) / 128), 128, 0, s>>>(
+  plan_kernel<<<static_cast<unsigned>((ntiles + kPlanWarps - 1) / kPlanWarps), 32 * kPlanWarps, 0, s>>>(
       rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, pp.cnt, pp.tiles);
   return cudaGetLastError();
 }
@@ -858,8 +892,8 @@ cudaError_t launch_tile_plan(const sla_block_lists& lists, int BH, int nrb, int 
   const int nt = rb == 128 ? nrb : (nrb + 1) / 2;
   const size_t ntiles = static_cast<size_t>(BH) * nt;
   if (ntiles == 0) return cudaSuccess;
-  plan_kernel<<<static_cast<unsigned>((ntiles + 127) / 128), 128, 0, s>>>(lists, BH, nrb, ncb, nt,
-                                                                          rb, cb, cnt, tiles);
+  plan_kernel<<<static_cast<unsigned>((ntiles + kPlanWarps - 1) / kPlanWarps), 32 * kPlanWarps, 0, s>>>(
+      lists, BH, nrb, ncb, nt, rb, cb, cnt, tiles);
   return cudaGetLastError();
 }
 
