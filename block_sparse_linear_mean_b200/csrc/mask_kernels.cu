@@ -802,14 +802,15 @@ cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
   }
   // top-k rows of up to 1024 blocks: one warp per row (measured faster than
   // the CTA kernel there, slower for rows of 1920 blocks); otherwise small
-  // CTAs for short rows (cheap barriers, many rows per SM), more threads per
-  // row for long ones
+  // CTAs for short rows and for CDF rows of up to 2048 blocks (cheap
+  // barriers, many rows per SM), more threads per row for long top-k rows
+  // (measured faster at 1920 blocks)
   const int nrows = g.BH * g.nqb;
   if (g.mode == SLA_MASK_TOPK && g.nkb <= 1024) {
     const int grid = (nrows + 7) / 8;
     if (g.nkb <= 512) classify_topk_warp_kernel<16><<<grid, 256, 0, s>>>(logits, a, nrows);
     else classify_topk_warp_kernel<32><<<grid, 256, 0, s>>>(logits, a, nrows);
-  } else if (g.nkb <= 1024) {
+  } else if (g.nkb <= 1024 || (g.mode == SLA_MASK_CDF && g.nkb <= 2048)) {
     if ((e = cudaFuncSetAttribute(classify_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(smem))) != cudaSuccess)
       return e;

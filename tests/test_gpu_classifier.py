@@ -40,7 +40,7 @@ def _params(nkb, nrows, mode, fc=0.0, fm=0.0, thr=0.0):
 @pytest.mark.parametrize("kind", ["dups", "zeros", "dyadic", "smooth"])
 # 1-512: one-warp top-k classifier with 16 blocks per lane, 700: 32 per lane,
 # 1920: the one-CTA classifier
-@pytest.mark.parametrize("nkb", [1, 7, 64, 300, 512, 700, 1920])
+@pytest.mark.parametrize("nkb", [1, 7, 64, 300, 512, 700, 1920, 2500])
 @pytest.mark.parametrize("mode,fc,fm,thr", [("topk", 0.05, 0.10, 0.0), ("topk", 0.5, 0.25, 0.0),
                                             ("cdf", 0.0, 0.0, 0.2), ("cdf", 0.0, 0.1, 0.5),
                                             ("cdf", 0.0, 0.0, 0.0)])
