@@ -27,12 +27,12 @@ namespace sla {
 // written split for the tf32 tensor-core logits: hi = tf32(m) in out and
 // lo = tf32(m - hi) in lo (m - hi is exact in fp32).
 template <typename T>
-__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, const T* __restrict__ xk,
+__global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ xq, const T* __restrict__ xk,
                                                    float* __restrict__ outq, float* __restrict__ outk,
                                                    float* __restrict__ loq, float* __restrict__ lok,
                                                    int N, int d, int bq, int bk) {
   constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
-  constexpr int kU = 4;                // loads in flight per thread
+  constexpr int kU = 8;                // loads in flight per thread
   const bool isk = blockIdx.z == 1;
   const int block = isk ? bk : bq, nb = (N + block - 1) / block;
   const int b = blockIdx.x, bh = blockIdx.y;
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ xq, con
       }
     }
   }
-  __shared__ float part[256 * 8];  // lanes * d <= 256 * VEC
+  __shared__ float part[128 * 8];  // lanes * d <= 128 * VEC
 #pragma unroll
   for (int e = 0; e < VEC; ++e) part[tl * d + v * VEC + e] = acc[e];
   __syncthreads();
@@ -97,11 +97,11 @@ cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, fl
                         float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s) {
   dim3 grid((N + min(bq, bk) - 1) / min(bq, bk), BH, 2);
   if (dtype == SLA_BF16)
-    pool_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
+    pool_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
                                                     static_cast<const __nv_bfloat16*>(k), qbar, kbar,
                                                     qlo, klo, N, d, bq, bk);
   else
-    pool_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+    pool_kernel<float><<<grid, 128, 0, s>>>(static_cast<const float*>(q), static_cast<const float*>(k),
                                             qbar, kbar, qlo, klo, N, d, bq, bk);
   return cudaGetLastError();
 }
