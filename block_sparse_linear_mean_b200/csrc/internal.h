@@ -30,8 +30,9 @@ constexpr double kFixedOne = 4611686018427387904.0;  // 2^62
 constexpr float kTieEps = 1e-5f;
 constexpr int kMaxBlocks = 8192;                     // Nqb, Nkb limit
 
-// TMA descriptors (tma_host.cu)
+// TMA descriptors and device queries (tma_host.cu)
 bool tma_available();
+int sm_count();
 bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box);
 bool encode_f32_map(void* map, const void* ptr, int rank, const uint64_t* dims,

@@ -677,15 +677,6 @@ cudaError_t set_smem(F kern, size_t bytes) {
 
 }  // namespace
 
-// SMs of the current device (one persistent CTA each)
-static int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    n = 148;
-  return n;
-}
-
 static cudaError_t launch_gather(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC,
                                  int ld, int nrow, int BH, int32_t* status, cudaStream_t s) {
   cudaError_t e;

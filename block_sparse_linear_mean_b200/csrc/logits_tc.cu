@@ -174,15 +174,6 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
   }
 }
 
-// SMs of the current device (one persistent CTA each)
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    n = 148;
-  return n;
-}
-
 }  // namespace
 
 bool logits_tc_supported(const Geom& g) {

@@ -1,5 +1,6 @@
 // Host-side TMA descriptor encoding (driver entry point looked up through the
-// runtime, so the library never links the driver directly).
+// runtime, so the library never links the driver directly), and the SM count
+// that sizes the persistent grids.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -20,6 +21,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool tma_available() { return encode_fn() != nullptr; }
+
+// SMs of the current device (persistent kernels launch one CTA per SM, or a
+// fixed number per SM); 148 if the query fails.
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
+}
 
 // Tensor of rank 2 or 3 (dims[0] innermost, strides in bytes for dims
 // 1..rank-1), 128-byte swizzle, out-of-range elements read as zero.

@@ -98,7 +98,8 @@ typedef struct {
   int32_t flags;             /* SLA_FLAG_* bits, 0 by default               */
 } sla_params;
 
-/* Force the portable fp32 SIMT kernels even for bf16 inputs (testing aid). */
+/* Force the portable fp32 SIMT kernels even for bf16 inputs, and the fp32
+ * FMA pooled logits (testing aid). */
 #define SLA_FLAG_SIMT 1
 /* Testing aid for the failure path: the tensor-core attention kernel's first
  * CTA withholds one K/V tile load and every bounded device-side wait gives up
@@ -138,7 +139,12 @@ SLA_API sla_status sla_workspace_size(const sla_params* p, int32_t op, size_t* b
  *   scores     [B,H,Nqb,Nkb] fp32 out, row-softmaxed pooled scores (nullable)
  *   tie_count  one int32 out (nullable): rows whose selection sits within
  *              1e-5 of a decision -- a score gap at a cut within 1e-5 of the
- *              higher score, or (CDF) a decisive tail sum within 1e-5 of thr */
+ *              higher score, or (CDF) a decisive tail sum within 1e-5 of thr
+ * The block means are fp32.  The pooled logits run on the tensor cores as
+ * three tf32 products per step (hi.hi + hi.lo + lo.hi of the means split as
+ * hi + lo), which keeps fp32 accuracy; SLA_FLAG_SIMT selects fp32 FMAs.  A
+ * device-side wait that times out on that path is reported by
+ * sla_check_device_status(ws) as SLA_ERR_TIMEOUT. */
 SLA_API sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
                           int8_t* mask, const sla_block_lists* rows,
                           const sla_block_lists* cols, float* scores,
