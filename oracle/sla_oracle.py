@@ -22,6 +22,10 @@ Sources (web pages on the method; they give words, not formulas):
 * The workload statement fixes phi = elu + 1 for the linear branch and a
   d x d output projection W applied to it, top-k fractions for the SLA split
   and the CDF rule for the NABLA split.
+* Veda article (mlllm.io, sections "Контекст" / context and the users'
+  section): a mask is judged by how well it reproduces dense attention,
+  max-pooled over tiles, and by its recall; the mask-quality functions at
+  the end follow it.
 
 Readings taken where the pages are silent (each is a plain choice, listed with
 its reason in the design notes and unpinned by the pages):
@@ -449,3 +453,62 @@ def backward(q, k, v, proj, mask, dout, block_q: int, block_k: int,
                 dk[b, h, a:e] += dpk * dphi(kj)
                 dv[b, h, a:e] += pk @ dh[j]
     return dict(dq=dq, dk=dk, dv=dv, dproj=dw)
+
+
+# --------------------------------------------------------------------------
+# mask quality: the selection against max-pooled dense attention
+#
+# Veda article (mlllm.io, section "Контекст" / context): what a block mask
+# has to reproduce is the structure of dense attention, and the reference
+# it is distilled toward is the dense attention max-pooled over tiles; the
+# article's user section reports the predictor's recall.  Below: the pooled
+# reference and the share of it a mask keeps.
+
+
+def max_pooled_attention(q, k, block_q: int, block_k: int,
+                         scale: Optional[float] = None) -> np.ndarray:
+    """Importance of (query block i, key block j): the largest dense softmax
+    probability between a real token of block i and a real key of block j,
+    each query token's softmax running over all N keys.
+    ``q, k [B, H, N, d] -> [B, H, Nqb, Nkb]``."""
+    q, k = f64(q), f64(k)
+    B, H, N, d = q.shape
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    nqb, nkb = n_blocks(N, block_q), n_blocks(N, block_k)
+    out = np.zeros((B, H, nqb, nkb))
+    for b in range(B):
+        for h in range(H):
+            logits = s * (q[b, h] @ k[b, h].T)                  # [N, N]
+            e = np.exp(logits - logits.max(axis=1, keepdims=True))
+            p = e / e.sum(axis=1, keepdims=True)
+            for i in range(nqb):
+                t0, t1 = block_range(i, N, block_q)
+                col_max = p[t0:t1].max(axis=0)                  # [N]
+                for j in range(nkb):
+                    s0, s1 = block_range(j, N, block_k)
+                    out[b, h, i, j] = col_max[s0:s1].max()
+    return out
+
+
+def mask_recall_counts(mask, importance) -> Tuple[int, int, int, int]:
+    """Per row (query block) with c critical blocks, the reference set is the
+    c blocks of largest importance (ties by lower index, the order of
+    reading 5); hits are the reference blocks the mask marks critical.  The
+    same with the kept set (critical or marginal) and its size.  Returns
+    (critical hits, critical total, kept hits, kept total) over all rows;
+    recall = hits / total."""
+    mask = np.asarray(mask)
+    imp = np.asarray(importance, dtype=np.float64)
+    nkb = mask.shape[-1]
+    m2 = mask.reshape(-1, nkb)
+    i2 = imp.reshape(-1, nkb)
+    ch = ct = kh = kt = 0
+    for row in range(m2.shape[0]):
+        order = rank_order(i2[row])
+        c = int((m2[row] == CRITICAL).sum())
+        ck = int((m2[row] != NEGLIGIBLE).sum())
+        ch += int((m2[row][order[:c]] == CRITICAL).sum())
+        kh += int((m2[row][order[:ck]] != NEGLIGIBLE).sum())
+        ct += c
+        kt += ck
+    return ch, ct, kh, kt
