@@ -57,6 +57,12 @@ cudaError_t launch_rows_from_mask(const int8_t* mask, const Geom& g,
 cudaError_t launch_cols_from_mask(const int8_t* mask, const Geom& g,
                                   const sla_block_lists& cols, cudaStream_t s);
 
+// mask quality (quality_kernels.cu)
+cudaError_t launch_block_importance(const void* q, const void* k, float* imp, const Geom& g,
+                                    cudaStream_t s);
+cudaError_t launch_mask_recall(const int8_t* mask, const float* imp, const Geom& g, int32_t* counts,
+                               cudaStream_t s);
+
 // forward
 cudaError_t launch_attn_simt(const void* q, const void* k, const void* v,
                              const Geom& g, const sla_block_lists& rows,

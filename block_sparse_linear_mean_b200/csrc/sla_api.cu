@@ -471,6 +471,29 @@ int32_t sla_forward_uses_tensor_cores(const sla_params* p) {
   return (g.dtype == SLA_BF16 && !(g.flags & SLA_FLAG_SIMT) && sla::attn_tc_supported(g)) ? 1 : 0;
 }
 
+sla_status sla_block_importance(const sla_params* p, const void* q, const void* k,
+                                float* importance, void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!q || !k || !importance || !aligned16(q) || !aligned16(k) || !aligned16(importance))
+    return SLA_ERR_INVALID_ARG;
+  SLA_CUDA(sla::launch_block_importance(q, k, importance, g, static_cast<cudaStream_t>(stream)));
+  return SLA_OK;
+}
+
+sla_status sla_mask_recall(const sla_params* p, const int8_t* mask, const float* importance,
+                           int32_t* counts, void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!mask || !importance || !counts || !aligned16(mask) || !aligned16(importance) ||
+      !aligned16(counts))
+    return SLA_ERR_INVALID_ARG;
+  SLA_CUDA(sla::launch_mask_recall(mask, importance, g, counts, static_cast<cudaStream_t>(stream)));
+  return SLA_OK;
+}
+
 sla_status sla_check_device_status(void* ws, void* stream) {
   if (!ws) return SLA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -42,6 +42,7 @@ EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",
            "sla_sparse_attention", "sla_sparse_attention_noalloc",
            "sla_linear_combine",
            "sla_backward", "sla_forward_uses_tensor_cores",
+           "sla_block_importance", "sla_mask_recall",
            "sla_check_device_status")
 
 
@@ -116,6 +117,10 @@ def lib():
                                    VP, VP, VP, VP, VP, SZ, VP]
         L.sla_forward_uses_tensor_cores.restype = ctypes.c_int32
         L.sla_forward_uses_tensor_cores.argtypes = [P(sla_params)]
+        L.sla_block_importance.restype = ctypes.c_int
+        L.sla_block_importance.argtypes = [P(sla_params), VP, VP, VP, VP]
+        L.sla_mask_recall.restype = ctypes.c_int
+        L.sla_mask_recall.argtypes = [P(sla_params), VP, VP, VP, VP]
         L.sla_check_device_status.restype = ctypes.c_int
         L.sla_check_device_status.argtypes = [VP, VP]
         _lib = L
@@ -209,6 +214,14 @@ def sla_forward_uses_tensor_cores(p: sla_params) -> int:
     return lib().sla_forward_uses_tensor_cores(ctypes.byref(p))
 
 
+def sla_block_importance(p, q, k, importance, stream) -> int:
+    return lib().sla_block_importance(ctypes.byref(p), q, k, importance, stream)
+
+
+def sla_mask_recall(p, mask, importance, counts, stream) -> int:
+    return lib().sla_mask_recall(ctypes.byref(p), mask, importance, counts, stream)
+
+
 def sla_check_device_status(ws, stream) -> int:
     return lib().sla_check_device_status(ws, stream)
 
@@ -294,6 +307,29 @@ def build_mask(p: sla_params, q: torch.Tensor, k: torch.Tensor, want_scores=Fals
                                             rc, cc, _ptr(scores), ties.data_ptr(),
                                             ws.data_ptr(), ws.numel(), _stream()))
     return dict(mask=mask, rows=rows, cols=cols, scores=scores, ties=ties[:1])
+
+
+def block_importance(p: sla_params, q: torch.Tensor, k: torch.Tensor) -> torch.Tensor:
+    """Dense attention max-pooled over (query block, key block) tiles,
+    ``[B,H,Nqb,Nkb]`` fp32 (a mask-quality measurement; dense work)."""
+    nqb, nkb = nblocks(p.N, p.block_q), nblocks(p.N, p.block_k)
+    imp = torch.empty(p.B, p.H, nqb, nkb, dtype=torch.float32, device=q.device)
+    _check("sla_block_importance", sla_block_importance(p, q.data_ptr(), k.data_ptr(),
+                                                        imp.data_ptr(), _stream()))
+    return imp
+
+
+def mask_recall(p: sla_params, mask: torch.Tensor, importance: torch.Tensor) -> dict:
+    """Recall of ``mask`` against ``importance``: hit and total counts for
+    the critical and the kept (critical or marginal) sets, and their
+    ratios (reads the four counts back to the host)."""
+    counts = torch.empty(4, dtype=torch.int32, device=mask.device)
+    _check("sla_mask_recall", sla_mask_recall(p, mask.data_ptr(), importance.data_ptr(),
+                                              counts.data_ptr(), _stream()))
+    ch, ct, kh, kt = (int(x) for x in counts.cpu().tolist())
+    return dict(critical_hits=ch, critical_total=ct, kept_hits=kh, kept_total=kt,
+                recall_critical=ch / ct if ct else float("nan"),
+                recall_kept=kh / kt if kt else float("nan"))
 
 
 def classify_scores(p: sla_params, scores: torch.Tensor, want_cols=False) -> dict:

@@ -271,6 +271,32 @@ SLA_API sla_status sla_backward(const sla_params* p, const void* q, const void* 
  * invalid.  Host only. */
 SLA_API int32_t sla_forward_uses_tensor_cores(const sla_params* p);
 
+/* Mask quality, step 1 (a measurement, not the hot path): dense attention
+ * max-pooled over (query block, key block) tiles -- the reference a block
+ * mask is judged against (Veda article, section "Контекст" / context).
+ *   q, k        [B,H,N,d] dtype, 16-byte aligned
+ *   importance  [B,H,Nqb,Nkb] fp32 out: for query block i and key block j,
+ *               the largest dense softmax probability between a real token
+ *               of block i and a real key of block j, each token's softmax
+ *               running over all N keys with p's scale
+ * Dense O(N^2 d) work on the SIMT cores, meant for N up to tens of
+ * thousands.  No workspace; asynchronous on `stream`. */
+SLA_API sla_status sla_block_importance(const sla_params* p, const void* q, const void* k,
+                                        float* importance, void* stream);
+
+/* Mask quality, step 2: recall of a mask against an importance map.
+ *   mask        [B,H,Nqb,Nkb] int8 in (2 critical, 1 marginal, 0 negligible)
+ *   importance  [B,H,Nqb,Nkb] fp32 in, non-negative
+ *   counts      4 int32 out, 16-byte aligned (set by the call): critical
+ *               hits, critical total, kept hits, kept total.  Per row with c
+ *               critical blocks the reference set is the c blocks of largest
+ *               importance (ties by lower block index); a hit is a reference
+ *               block the mask marks critical.  "Kept" does the same with the
+ *               critical-or-marginal set.  recall = hits / total.
+ * Asynchronous on `stream`. */
+SLA_API sla_status sla_mask_recall(const sla_params* p, const int8_t* mask,
+                                   const float* importance, int32_t* counts, void* stream);
+
 /* Synchronises `stream` and returns the status word the last call on `ws`
  * left (SLA_OK, or SLA_ERR_TIMEOUT when a bounded device-side wait gave up),
  * or SLA_ERR_CUDA when a CUDA error is pending. */
