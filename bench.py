@@ -63,7 +63,33 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mask-quality", action="store_true",
+                    help="instead of the timed step: recall of the workload's mask against "
+                         "the dense attention max-pooled over tiles (one GPU; dense work)")
     return ap.parse_args()
+
+
+def run_mask_quality(args):
+    """Mask quality on the workload (one GPU): the pooled-score mask against
+    the dense attention max-pooled over (query block, key block) tiles, both
+    from the library's kernels.  Prints one JSON line."""
+    from block_sparse_linear_mean_b200 import sla
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    x = synth.make_inputs(wl, seed=0, device=dev)
+    p = sla.params_for(wl)
+    m = sla.build_mask(p, x.q, x.k)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    imp = sla.block_importance(p, x.q, x.k)
+    e1.record()
+    rec = sla.mask_recall(p, m["mask"], imp)
+    return {"workload": wl.name, "config": wl.description,
+            "mask_quality": {"reference": "dense attention max-pooled over (query block, key block) "
+                                          "tiles; per row as many reference blocks as the mask keeps",
+                             **{k: (round(v, 4) if isinstance(v, float) else v) for k, v in rec.items()},
+                             "importance_ms": round(e0.elapsed_time(e1), 2)}}
 
 
 def load_peaks():
@@ -545,6 +571,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.mask_quality:
+        if rank == 0:
+            print(json.dumps(run_mask_quality(args)))
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:
