@@ -33,6 +33,8 @@ SLA_MASK_TOPK, SLA_MASK_CDF = 0, 1
 SLA_OP_MASK, SLA_OP_FORWARD, SLA_OP_BACKWARD = 0, 1, 2
 SLA_FLAG_SIMT = 1
 SLA_FLAG_DEBUG_TIMEOUT = 2
+# block labels in the int8 mask
+CRITICAL, MARGINAL, NEGLIGIBLE = 2, 1, 0
 
 # Entry points declared in include/sla.h (checked by the test-suite).
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",
@@ -330,6 +332,30 @@ def mask_recall(p: sla_params, mask: torch.Tensor, importance: torch.Tensor) -> 
     return dict(critical_hits=ch, critical_total=ct, kept_hits=kh, kept_total=kt,
                 recall_critical=ch / ct if ct else float("nan"),
                 recall_kept=kh / kt if kt else float("nan"))
+
+
+def flex_block_mask(p: sla_params, mask: torch.Tensor, rows: BlockLists):
+    """The critical part of a block mask as a PyTorch Flex Attention
+    ``BlockMask`` (NABLA post, SberAIScience channel: the method is fully
+    compatible with PyTorch's Flex Attention).  ``kv_num_blocks`` and
+    ``kv_indices`` are zero-copy views of the CSR lists (``[B,H,Nqb]``
+    counts, ``[B,H,Nqb,Nkb]`` ascending critical key blocks); the block
+    sizes are (block_q, block_k); the sequence length N covers the ragged
+    tail; the ``mask_mod`` reads the int8 mask (critical = 2), so every Flex
+    path, the eager one included, attends to the critical blocks only.  The
+    marginal (linear) branch has no Flex counterpart and is not exported.
+    ``mask`` must outlive the returned object."""
+    from torch.nn.attention.flex_attention import BlockMask
+    nqb, nkb = nblocks(p.N, p.block_q), nblocks(p.N, p.block_k)
+    bq, bk = p.block_q, p.block_k
+    kv_num = rows.crit_cnt.view(p.B, p.H, nqb)
+    kv_idx = rows.crit_idx.view(p.B, p.H, nqb, nkb)
+
+    def critical(b, h, q_idx, kv_idx):
+        return mask[b, h, q_idx // bq, kv_idx // bk] == CRITICAL
+
+    return BlockMask.from_kv_blocks(kv_num, kv_idx, BLOCK_SIZE=(bq, bk), mask_mod=critical,
+                                    seq_lengths=(p.N, p.N))
 
 
 def classify_scores(p: sla_params, scores: torch.Tensor, want_cols=False) -> dict:
