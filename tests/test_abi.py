@@ -135,6 +135,8 @@ def test_null_pointers_rejected_before_any_cuda_call(lib):
                             None, None, None, None, None, None, 0,
                             None) == sla.SLA_ERR_INVALID_ARG
     assert sla.sla_mask_lists(p, None, None, None, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_block_importance(p, None, None, None, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_mask_recall(p, None, None, None, None) == sla.SLA_ERR_INVALID_ARG
     assert sla.sla_check_device_status(None, None) == sla.SLA_ERR_INVALID_ARG
 
 
@@ -145,6 +147,18 @@ def test_misaligned_pointer_rejected(lib):
     lists = sla.sla_block_lists(16, 16, 16, 16)
     st = sla.sla_build_mask(p, 16, 24, 16, lists, None, None, None, 16, 1 << 40, None)
     assert st == sla.SLA_ERR_INVALID_ARG
+
+
+def test_mask_quality_entry_points_validate_on_the_host(lib):
+    p = good_params()
+    # misaligned (never dereferenced) addresses
+    assert sla.sla_block_importance(p, 16, 24, 16, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_mask_recall(p, 16, 16, 20, None) == sla.SLA_ERR_INVALID_ARG
+    # an invalid parameter block is refused before the pointers are looked at
+    bad = good_params()
+    bad.d = 96
+    assert sla.sla_block_importance(bad, 16, 16, 16, None) == sla.SLA_ERR_UNSUPPORTED
+    assert sla.sla_mask_recall(bad, 16, 16, 16, None) == sla.SLA_ERR_UNSUPPORTED
 
 
 def test_workspace_too_small_rejected(lib):
