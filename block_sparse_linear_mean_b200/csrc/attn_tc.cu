@@ -80,6 +80,9 @@ __device__ __forceinline__ uint32_t entry(int blk, uint32_t flags) {
 // membership flags whatever the lists' order; entries outside [0, nkb) are
 // skipped and repeated entries collapse.
 constexpr int kPlanWarps = 4;
+// (parameter validation caps Nqb and Nkb at kMaxBlocks: the bitmaps below
+// hold that many blocks and an entry's index field has 13 bits)
+static_assert(kMaxBlocks <= 8192, "plan entries hold 13-bit block indices");
 
 __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(sla_block_lists rows, int BH, int nqb,
                                                                int nkb, int nqt, int bq, int bk,

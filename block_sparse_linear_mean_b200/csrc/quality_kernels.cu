@@ -17,7 +17,8 @@
 //                            (critical or marginal) set
 //
 // The importance is dense O(N^2 d) work on the SIMT cores, meant for N up to
-// tens of thousands.
+// tens of thousands; the recall ranks each row's blocks by counting, O(Nkb^2)
+// per row.
 #include <float.h>
 
 #include "common.cuh"

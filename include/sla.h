@@ -293,7 +293,7 @@ SLA_API sla_status sla_block_importance(const sla_params* p, const void* q, cons
  *               importance (ties by lower block index); a hit is a reference
  *               block the mask marks critical.  "Kept" does the same with the
  *               critical-or-marginal set.  recall = hits / total.
- * Asynchronous on `stream`. */
+ * O(Nkb^2) comparisons per row.  Asynchronous on `stream`. */
 SLA_API sla_status sla_mask_recall(const sla_params* p, const int8_t* mask,
                                    const float* importance, int32_t* counts, void* stream);
 
