@@ -92,6 +92,23 @@ def run_mask_quality(args):
                              "importance_ms": round(e0.elapsed_time(e1), 2)}}
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's milliseconds, on every rank (one all-reduce); the
+    value itself on a single process."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, flops_per_step: float, steps: int, ms: float) -> float:
+    """Whole-job TFLOP/s: each of the `world` ranks ran `steps` steps of its
+    own problem within `ms` milliseconds (the slowest rank's time)."""
+    return world * flops_per_step * steps / (ms * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -368,13 +385,9 @@ def run_ours(args, rank, world, local_rank):
     t_prep = [e[1].elapsed_time(e[2]) for e in ev]
     t_comb = [e[2].elapsed_time(e[3]) for e in ev]
     t_bwd = [e[3].elapsed_time(e[4]) for e in ev]
-    total_ms = sum(e[0].elapsed_time(e[4]) for e in ev)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[4]) for e in ev), dev)
     ms_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_rate(world, flops, args.steps, total_ms)
 
     # end to end through the C ABI with host buffers: every step copies its
     # inputs (q, k, v, and dO for the fine-tune step) from pinned host memory,
@@ -432,12 +445,8 @@ def run_ours(args, rank, world, local_rank):
         ds.wait_event(ev_comp[args.steps - 1])
         t1.record(ds)
         torch.cuda.synchronize(dev)
-        e2e_ms = t0.elapsed_time(t1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), dev)
+        e2e = {"value": job_rate(world, flops, args.steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in ins)),
                "d2h_bytes_per_step": int(out.numel() * out.element_size() +
                                          sum(t.numel() * t.element_size() for t in gsrc)),
