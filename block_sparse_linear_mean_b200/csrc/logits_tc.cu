@@ -8,9 +8,11 @@
 // The means arrive split as m = hi + lo with hi = tf32(m), lo = tf32(m - hi)
 // (the pooling kernel writes both), and each product is taken as
 //   lo_q . hi_k + hi_q . lo_k + hi_q . hi_k
-// with kind::tf32 MMAs accumulating in fp32 tensor memory.  The dropped
-// lo . lo term and the rounding of lo are below 2^-21 of |q| |k| per channel,
-// about the size of fp32 rounding, so the logits carry fp32 accuracy.
+// with kind::tf32 MMAs accumulating in fp32 tensor memory.  With |m - hi| <=
+// 2^-11 |m| and |(m - hi) - lo| <= 2^-22 |m|, the dropped lo . lo term and
+// the rounding of lo stay below 3 * 2^-22 (under 2^-20) of |q| |k| per
+// channel, about the size of fp32 rounding, so the logits carry fp32
+// accuracy.
 //
 // Persistent kernel, one CTA per SM, 128 x 128 output tiles (query blocks x
 // key blocks) walked in (m, n, bh) order:
