@@ -512,3 +512,29 @@ def mask_recall_counts(mask, importance) -> Tuple[int, int, int, int]:
         ct += c
         kt += ck
     return ch, ct, kh, kt
+
+
+# --------------------------------------------------------------------------
+# token order in 3D tiles
+#
+# Veda article (mlllm.io, sections "Что произошло" / what happened and
+# "Контекст" / context): attention is selected over tiles of tokens, with
+# tile shapes fitted per head and layer.  Blocks of consecutive tokens then
+# cover compact spatio-temporal boxes instead of raster strips.
+
+
+def tile_order(grid: Tuple[int, int, int], tile: Tuple[int, int, int]) -> np.ndarray:
+    """Token order of 3D tiles over a raster grid (F, R, C), token
+    t = (f R + r) C + c: tiles in raster order over the tile grid, tokens in
+    raster order inside each tile, tiles at the far edges partial.  Returns
+    ``perm`` with ``perm[n]`` = raster index of the n-th token in tile order
+    (``x[..., perm, :]`` reorders a ``[..., N, d]`` tensor)."""
+    F, R, C = grid
+    tf, tr, tc = tile
+    idx = np.arange(F * R * C).reshape(F, R, C)
+    parts = []
+    for f0 in range(0, F, tf):
+        for r0 in range(0, R, tr):
+            for c0 in range(0, C, tc):
+                parts.append(idx[f0:f0 + tf, r0:r0 + tr, c0:c0 + tc].reshape(-1))
+    return np.concatenate(parts)
