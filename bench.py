@@ -183,7 +183,8 @@ def backward_flops(wl, mask_np):
 class ClockSampler:
     """Samples SM clock and clock-event (throttle) reasons of one GPU every
     20 ms through NVML in a background thread while the timed region runs;
-    raw samples go to gpurun_out/clocks_rank<i>.csv."""
+    the raw samples are written as CSV, one file per rank, beside the other
+    run outputs."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
                "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}

@@ -1,7 +1,7 @@
 // Mask quality: how much of dense attention a block mask keeps.
 //
 // Veda article (mlllm.io, section "Контекст" / context): a sparsity mask is
-// judged by how well it reproduces the structure of dense attention, and the
+// evaluated by how well it reproduces the structure of dense attention, and the
 // reference its predictor is distilled toward is the dense attention
 // max-pooled over tiles; the article's users' section reports the
 // predictor's recall.  Two measurement kernels (not on the hot path):

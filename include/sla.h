@@ -273,7 +273,7 @@ SLA_API int32_t sla_forward_uses_tensor_cores(const sla_params* p);
 
 /* Mask quality, step 1 (a measurement, not the hot path): dense attention
  * max-pooled over (query block, key block) tiles -- the reference a block
- * mask is judged against (Veda article, section "Контекст" / context).
+ * mask is evaluated against (Veda article, section "Контекст" / context).
  *   q, k        [B,H,N,d] dtype, 16-byte aligned
  *   importance  [B,H,Nqb,Nkb] fp32 out: for query block i and key block j,
  *               the largest dense softmax probability between a real token

@@ -23,7 +23,7 @@ Sources (web pages on the method; they give words, not formulas):
   d x d output projection W applied to it, top-k fractions for the SLA split
   and the CDF rule for the NABLA split.
 * Veda article (mlllm.io, sections "Контекст" / context and the users'
-  section): a mask is judged by how well it reproduces dense attention,
+  section): a mask is evaluated by how well it reproduces dense attention,
   max-pooled over tiles, and by its recall; the mask-quality functions at
   the end follow it.
 
