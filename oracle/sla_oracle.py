@@ -27,8 +27,10 @@ Sources (web pages on the method; they give words, not formulas):
   max-pooled over tiles, and by its recall; the mask-quality functions at
   the end follow it.
 
-Readings taken where the pages are silent (each is a plain choice, listed with
-its reason in the design notes and unpinned by the pages):
+Readings taken where the pages are silent.  Each is the plainest choice the
+rest of the pages support; readings 1, 4 (the rounding of the counts), 5 (the
+index tie-break) and the diagonal block not being forced critical are
+conventions the pages do not fix, so no page value pins them:
 
 1. A block that ends at N (ragged tail) is pooled over its real tokens only.
 2. Scores and attention use the scale s = 1/sqrt(d) unless a scale is given.
