@@ -48,12 +48,6 @@ constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 3;
 constexpr int kSBuf = 2;  // S tiles in TMEM, one per warpgroup (P overwrites its S)
-// One pair in kPolyEvery of a full tile's exponentials is computed by a cubic
-// on the FMA pipe instead of the special-function unit (0: none).  Here the
-// softmax warp is bound by latency rather than by the special-function
-// unit, and the cubic's extra instructions cost more than they save.
-constexpr int kPolyEvery = 0;
-constexpr int kPolyStep = kPolyEvery > 0 ? kPolyEvery : 1;
 constexpr int kSoftmaxWarps = 8;                 // two warpgroups
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;  // TMA warp, MMA warp, softmax
 constexpr uint32_t kSmemRequest = 232448;          // 227 KB opt-in maximum
@@ -531,8 +525,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // exponentials of the loaded half (kv of its 64 keys valid) as bf16
       // pairs into pk[0, 32), the sum of those rounded weights -- the ones
       // P V uses, so O / l is a convex combination of V rows -- into acc;
-      // returns the max of the valid raw scores.  Every kPolyEvery-th pair of
-      // a full half goes to the FMA pipe.
+      // returns the max of the valid raw scores.
       auto half_exp = [&](int kv, uint32_t* pk) -> float {
         const float2 sc2 = make_float2(scale_log2, scale_log2);
         const float2 nm2 = make_float2(-m_ref, -m_ref);
@@ -544,9 +537,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (i & 1) a1 = max3(a1, s[2 * i], s[2 * i + 1]);
             else a0 = max3(a0, s[2 * i], s[2 * i + 1]);
             const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sc2, nm2);
-            const float2 ex = (kPolyEvery > 0 && i % kPolyStep == kPolyEvery - 1)
-                                  ? exp2_poly2(x)
-                                  : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            const float2 ex = make_float2(fast_exp2(x.x), fast_exp2(x.y));
             pk[i] = pack_bf16x2(ex.x, ex.y);
             if (i % 4 == 0) add_bf16x2_f32(pk[i], acc0.x, acc0.y);
             if (i % 4 == 1) add_bf16x2_f32(pk[i], acc1.x, acc1.y);
@@ -845,10 +836,9 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                                        static_cast<int>(kSmemRequest));
   if (e != cudaSuccess) return e;
   const float scale_log2 = g.scale * 1.4426950408889634f;
-  const bool debug = (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0;
-  const long long timeout = debug ? (1ll << 24) : (1ll << 31);
+  const int debug_skip = debug_withhold(g, SLA_WITHHOLD_ATTENTION) ? 1 : 0;
   kern<<<g.BH * nqt, kThreads, kSmemRequest, s>>>(mq, mk, mv, mhm, mw, mo, cnt, tiles, g.nkb, ep, status,
-                                                  g.N, nqt, scale_log2, timeout, debug ? 1 : 0);
+                                                  g.N, nqt, scale_log2, wait_limit(g), debug_skip);
   return cudaGetLastError();
 }
 

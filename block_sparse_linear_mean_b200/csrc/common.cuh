@@ -49,6 +49,14 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
 __device__ __forceinline__ float dphi(float x) { return x > 0.f ? 1.f : expf(x); }
 
+// ---------------------------------------------------------------- scores
+// A non-negative fp32 score (given as its bit pattern) in 2^-62 fixed point,
+// truncated: exact for scores above 2^-39, and sums of such values are
+// exact and independent of their order (integer adds).
+__device__ __forceinline__ uint64_t to_fixed(uint32_t pbits) {
+  return __double2ull_rz(static_cast<double>(__uint_as_float(pbits)) * kFixedOne);
+}
+
 // ---------------------------------------------------------------- warps
 
 __device__ __forceinline__ float warp_sum(float v) {

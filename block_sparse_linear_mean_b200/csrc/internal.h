@@ -26,12 +26,24 @@ struct Geom {
   bool linear;         // linear branch on (frac_marg > 0)
 };
 
+// Bounded device-side waits give up after this many cycles (~1.1 s at
+// 1.965 GHz; ~8.5 ms under SLA_FLAG_DEBUG_TIMEOUT).
+inline long long wait_limit(const Geom& g) {
+  return (g.flags & SLA_FLAG_DEBUG_TIMEOUT) ? (1ll << 24) : (1ll << 31);
+}
+// Testing aid: true when kernel `k` (sla_withhold_kernel) is the one whose
+// first CTA withholds a tile load under SLA_FLAG_DEBUG_TIMEOUT.
+inline bool debug_withhold(const Geom& g, int k) {
+  return (g.flags & SLA_FLAG_DEBUG_TIMEOUT) != 0 && ((g.flags >> 8) & 0xF) == k;
+}
+
 constexpr double kFixedOne = 4611686018427387904.0;  // 2^62
 constexpr float kTieEps = 1e-5f;
 constexpr int kMaxBlocks = 8192;                     // Nqb, Nkb limit
 
 // TMA descriptors and device queries (tma_host.cu)
 bool tma_available();
+bool current_context_id(unsigned long long* id);
 int sm_count();
 bool encode_bf16_map(void* map, const void* ptr, int rank, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box);
@@ -163,7 +175,7 @@ LinInputs lin_tc_inputs(const Geom& g, void* scratch, const sla_block_lists& row
 // BH * nrow * ld bf16 (ld = ncol rounded up to 64).
 cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, int ncol,
                                const void* src_h, const float* src_z, void* dst_h, float* dst_z,
-                               void* ind, int ld, int32_t* status, cudaStream_t s);
+                               void* ind, int ld, int32_t* status, const Geom& g, cudaStream_t s);
 
 // backward of the linear branch and the projection on the tensor cores
 // (lin_bwd_tc.cu): dq, dk, dv are added to; dproj is written.

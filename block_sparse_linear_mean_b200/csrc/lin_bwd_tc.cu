@@ -259,7 +259,7 @@ cudaError_t launch_lin_bwd_gather(const sla_block_lists& cols, const Geom& g, vo
   // without marginal sets)
   cudaError_t e = launch_list_gather(cols, g.BH, g.nkb, g.nqb, sc + w.dhm,
                                      reinterpret_cast<const float*>(sc + w.dzm), sc + w.dh,
-                                     reinterpret_cast<float*>(sc + w.dz), sc + w.indt, w.ldt, status, s);
+                                     reinterpret_cast<float*>(sc + w.dz), sc + w.indt, w.ldt, status, g, s);
   if (e != cudaSuccess) return e;
   lin->dh = sc + w.dh;
   lin->dz = reinterpret_cast<const float*>(sc + w.dz);

@@ -24,7 +24,6 @@ namespace sla {
 
 namespace {
 
-constexpr long long kTimeout = 1ll << 31;
 constexpr int kD = 128;
 constexpr int kHElems = kD * kD;  // 16384
 
@@ -48,7 +47,7 @@ template <int BK>
 __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __grid_constant__ CUtensorMap tmH, float* __restrict__ zsum, int N, int nkb,
-    int32_t* status) {
+    int32_t* status, long long timeout, int debug_skip) {
   constexpr uint32_t kChunk = BK * 128;  // bytes of one 64-column chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
@@ -69,14 +68,15 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  if (tid == 0) {
+  // (test aid: the first CTA's tiles never arrive)
+  if (tid == 0 && !(debug_skip && blockIdx.x == 0 && blockIdx.y == 0)) {
     mbar_expect_tx(b_tma, 4 * kChunk);
     for (int c = 0; c < 2; ++c) {
       tma_load_3d(sb + offK + c * kChunk, &tmK, c * 64, j * BK, bh, b_tma);
       tma_load_3d(sb + offV + c * kChunk, &tmV, c * 64, j * BK, bh, b_tma);
     }
   }
-  bool ok = __syncthreads_and(wait_bounded(b_tma, 0, status, kTimeout));
+  bool ok = __syncthreads_and(wait_bounded(b_tma, 0, status, timeout));
   if (ok) {
     for (int x = tid; x < BK * 16; x += 128) {
       const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
                idesc, kk > 0);
       tc_commit(b_mma);
     }
-    ok = __syncthreads_and(wait_bounded(b_mma, 0, status, kTimeout));
+    ok = __syncthreads_and(wait_bounded(b_mma, 0, status, timeout));
   }
   if (ok) {  // TMEM lane a -> bf16 row a of a 128B-swizzled staging tile (reuses K/V space)
     tc_fence_after();
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
 __global__ void __launch_bounds__(128) lin_summary_persist_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __grid_constant__ CUtensorMap tmH, float* __restrict__ zsum, int N, int nkb, int nitems,
-    int32_t* status) {
+    int32_t* status, long long timeout, int debug_skip) {
   constexpr int BK = 64;
   constexpr uint32_t kChunk = BK * 128;  // bytes of one 64-column chunk
   constexpr uint32_t kBuf = 4 * kChunk;  // K (2 chunks) then V (2 chunks); 32 KB = one H tile
@@ -193,7 +193,9 @@ __global__ void __launch_bounds__(128) lin_summary_persist_kernel(
       tma_load_3d(dst + 2 * kChunk + c * kChunk, &tmV, c * 64, j * BK, bh, b_tma(b));
     }
   };
-  if (tid == 0 && static_cast<int>(blockIdx.x) < nitems) issue_load(blockIdx.x, 0);
+  // (test aid: the first CTA's first item never arrives)
+  if (tid == 0 && static_cast<int>(blockIdx.x) < nitems && !(debug_skip && blockIdx.x == 0))
+    issue_load(blockIdx.x, 0);
   bool ok = true;
   int k = 0;
   for (int w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++k) {
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(128) lin_summary_persist_kernel(
       tma_store_wait_read();
       issue_load(w + gridDim.x, b ^ 1);
     }
-    ok = __syncthreads_and(wait_bounded(b_tma(b), (k >> 1) & 1, status, kTimeout));
+    ok = __syncthreads_and(wait_bounded(b_tma(b), (k >> 1) & 1, status, timeout));
     if (!ok) break;
     for (int x = tid; x < BK * 16; x += 128) {
       const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(128) lin_summary_persist_kernel(
                idesc, kk > 0);
       tc_commit(b_mma);
     }
-    ok = __syncthreads_and(wait_bounded(b_mma, k & 1, status, kTimeout));
+    ok = __syncthreads_and(wait_bounded(b_mma, k & 1, status, timeout));
     if (!ok) break;
     // TMEM lane a -> bf16 row a of a 128B-swizzled staging tile (this buffer)
     tc_fence_after();
@@ -359,7 +361,7 @@ constexpr size_t kGSmem = kGBars + 256 + 1024;
 __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const __grid_constant__ CUtensorMap tmC, int ksteps, int tiles_m, int tiles_n, int ntiles,
-    int32_t* status) {
+    int32_t* status, long long timeout, int debug_skip) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const uint32_t sb = smem_u32(base);
@@ -396,8 +398,9 @@ __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
       coords(t, m0, n0, bh);
       for (int ks = 0; ks < ksteps && ok; ++ks, ++g) {
         const int s = g % kGStages;
-        if (g >= kGStages) ok = wait_bounded(b_empty(s), ((g / kGStages) & 1) ^ 1, status, kTimeout);
+        if (g >= kGStages) ok = wait_bounded(b_empty(s), ((g / kGStages) & 1) ^ 1, status, timeout);
         if (!ok) break;
+        if (debug_skip && blockIdx.x == 0 && g == 0) continue;  // test aid: this step never arrives
         const uint32_t st = sb + s * kGStage;
         mbar_expect_tx(b_full(s), kGStage);
         tma_load_3d(st, &tmA, ks * 64, m0, bh, b_full(s));
@@ -412,10 +415,10 @@ __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
       const int a = it & 1;
       // the epilogue has drained this accumulator (tile it - 2)
-      if (it >= 2) ok = wait_bounded(b_acc_empty(a), ((it >> 1) & 1) ^ 1, status, kTimeout);
+      if (it >= 2) ok = wait_bounded(b_acc_empty(a), ((it >> 1) & 1) ^ 1, status, timeout);
       for (int ks = 0; ks < ksteps && ok; ++ks, ++g) {
         const int s = g % kGStages;
-        ok = wait_bounded(b_full(s), (g / kGStages) & 1, status, kTimeout);
+        ok = wait_bounded(b_full(s), (g / kGStages) & 1, status, timeout);
         if (!ok) break;
         tc_fence_after();
         const uint32_t so = s * kGStage;
@@ -435,7 +438,7 @@ __global__ void __launch_bounds__(192, 1) gather_gemm_kernel(
       const int a = it & 1;
       int m0, n0, bh;
       coords(t, m0, n0, bh);
-      ok = wait_bounded(b_acc_full(a), (it >> 1) & 1, status, kTimeout);
+      ok = wait_bounded(b_acc_full(a), (it >> 1) & 1, status, timeout);
       tc_fence_after();
       for (int hf = 0; hf < 2; ++hf) {  // (every warp reaches the barrier below)
         // the previous stores have read the staging half tile
@@ -495,7 +498,7 @@ __global__ void __launch_bounds__(128) lin_apply_tc_kernel(
     const __grid_constant__ CUtensorMap tmHM, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmW, const float* __restrict__ zmar,
     sla_block_lists rows, const float* __restrict__ o_s, __nv_bfloat16* __restrict__ out,
-    float* __restrict__ o_lin, int N, int nqb, int nkb, int32_t* status) {
+    float* __restrict__ o_lin, int N, int nqb, int nkb, int32_t* status, long long timeout) {
   constexpr uint32_t offHM = 0, offW = 32768, offQ = 65536;
   constexpr uint32_t kQChunk = BQ * 128;
   constexpr uint32_t offOL = offQ + 2 * kQChunk;      // BQ/64 chunks of [128 a][64 t]
@@ -541,7 +544,7 @@ __global__ void __launch_bounds__(128) lin_apply_tc_kernel(
       tma_load_3d(sb + offQ + kQChunk, &tmQ, 64, t0g, bh, b_tma);
     }
     zm[c] = zmar[i64(list_row) * kD + c];  // z^M, gathered by the indicator kernel
-    ok = __syncthreads_and(wait_bounded(b_tma, 0, status, kTimeout));
+    ok = __syncthreads_and(wait_bounded(b_tma, 0, status, timeout));
     if (ok) {
       for (int x = tid; x < BQ * 16; x += 128) {  // phi(Q) in place, padding rows zero
         const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
@@ -566,7 +569,7 @@ __global__ void __launch_bounds__(128) lin_apply_tc_kernel(
                  sdesc(sb + offQ + (kk >> 2) * kQChunk + (kk & 3) * 32, 16, 1024), idesc, kk > 0);
         tc_commit(b_m1);
       }
-      ok = __syncthreads_and(wait_bounded(b_m1, 0, status, kTimeout));
+      ok = __syncthreads_and(wait_bounded(b_m1, 0, status, timeout));
     }
     if (ok) {
       tc_fence_after();
@@ -601,7 +604,7 @@ __global__ void __launch_bounds__(128) lin_apply_tc_kernel(
                  sdesc(sb + offOL + kk * 2048, 16384, 1024), idesc, kk > 0);
         tc_commit(b_m2);
       }
-      ok = __syncthreads_and(wait_bounded(b_m2, 0, status, kTimeout));
+      ok = __syncthreads_and(wait_bounded(b_m2, 0, status, timeout));
     }
     if (ok) {
       tc_fence_after();
@@ -678,13 +681,16 @@ cudaError_t set_smem(F kern, size_t bytes) {
 }  // namespace
 
 static cudaError_t launch_gather(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC,
-                                 int ld, int nrow, int BH, int32_t* status, cudaStream_t s) {
+                                 int ld, int nrow, int BH, int32_t* status, const Geom& geo,
+                                 cudaStream_t s) {
   cudaError_t e;
   if ((e = set_smem(gather_gemm_kernel, kGSmem)) != cudaSuccess) return e;
   const int tiles_m = (nrow + 127) / 128, tiles_n = kHElems / 256;
   const int ntiles = tiles_m * tiles_n * BH;
   const int grid = std::min(ntiles, sm_count());
-  gather_gemm_kernel<<<grid, 192, kGSmem, s>>>(mA, mB, mC, ld / 64, tiles_m, tiles_n, ntiles, status);
+  gather_gemm_kernel<<<grid, 192, kGSmem, s>>>(mA, mB, mC, ld / 64, tiles_m, tiles_n, ntiles, status,
+                                               wait_limit(geo),
+                                               debug_withhold(geo, SLA_WITHHOLD_GATHER) ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -712,7 +718,8 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
 
 cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, int ncol,
                                const void* src_h, const float* src_z, void* dst_h, float* dst_z,
-                               void* ind, int ld, int32_t* status, cudaStream_t s) {
+                               void* ind, int ld, int32_t* status, const Geom& g,
+                               cudaStream_t s) {
   cudaError_t e;
   uint16_t* indp = static_cast<uint16_t*>(ind);
   indicator_kernel<<<BH * nrow, 128, 0, s>>>(lists, indp, src_z, dst_z, nrow, ncol, ld);
@@ -728,7 +735,7 @@ cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, i
   if (!encode_bf16_map(&mA, indp, 3, da, sa, ba) || !encode_bf16_map(&mB, src_h, 3, db, sbt, bb) ||
       !encode_bf16_map(&mC, dst_h, 3, dc, sc2, bc))
     return cudaErrorInvalidValue;
-  return launch_gather(mA, mB, mC, ld, nrow, BH, status, s);
+  return launch_gather(mA, mB, mC, ld, nrow, BH, status, g, s);
 }
 
 cudaError_t launch_lin_tc_prepare(const void* k, const void* v, const float* proj,
@@ -797,6 +804,7 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 1. summaries
   {
+    const int debug_skip = debug_withhold(g, SLA_WITHHOLD_SUMMARIES) ? 1 : 0;
     // at least 48 KB so at most 4 CTAs share an SM: 4 x 128 TMEM columns fit
     const size_t smem = std::max<size_t>(4 * size_t(g.bk) * 128 + 64 + 1024, 48 * 1024);
     dim3 grid(g.nkb, g.BH);
@@ -807,17 +815,19 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
       if ((e = set_smem(lin_summary_persist_kernel, psmem)) != cudaSuccess) return e;
       const int nitems = g.BH * g.nkb;
       const int pgrid = std::min(nitems, 3 * sm_count());
-      lin_summary_persist_kernel<<<pgrid, 128, psmem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, nitems, status);
+      lin_summary_persist_kernel<<<pgrid, 128, psmem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, nitems, status,
+                                                           wait_limit(g), debug_skip);
     } else {
       if ((e = set_smem(lin_summary_tc_kernel<128>, smem)) != cudaSuccess) return e;
-      lin_summary_tc_kernel<128><<<grid, 128, smem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, status);
+      lin_summary_tc_kernel<128><<<grid, 128, smem, s>>>(mK, mV, mH, zbuf, g.N, g.nkb, status,
+                                                         wait_limit(g), debug_skip);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 2. indicator + gather GEMM
   indicator_kernel<<<g.BH * g.nqb, 128, 0, s>>>(rows, ind, zbuf, zmbuf, g.nqb, g.nkb, w.ld);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = launch_gather(mA, mB, mC, w.ld, g.nqb, g.BH, status, s)) != cudaSuccess) return e;
+  if ((e = launch_gather(mA, mB, mC, w.ld, g.nqb, g.BH, status, g, s)) != cudaSuccess) return e;
   }  // prepare
   // 3-4. apply + combine
   if (apply) {
@@ -827,12 +837,12 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
       const size_t smem = 65536 + 2 * 64 * 128 + 16384 + 512 + 256 + 64 + 1024;
       if ((e = set_smem(lin_apply_tc_kernel<64>, smem)) != cudaSuccess) return e;
       lin_apply_tc_kernel<64><<<grid, 128, smem, s>>>(mHM, mQ, mW, zmbuf, rows, o_s, ob, o_lin, g.N,
-                                                      g.nqb, g.nkb, status);
+                                                      g.nqb, g.nkb, status, wait_limit(g));
     } else {
       const size_t smem = 65536 + 2 * 128 * 128 + 32768 + 512 + 512 + 64 + 1024;
       if ((e = set_smem(lin_apply_tc_kernel<128>, smem)) != cudaSuccess) return e;
       lin_apply_tc_kernel<128><<<grid, 128, smem, s>>>(mHM, mQ, mW, zmbuf, rows, o_s, ob, o_lin, g.N,
-                                                       g.nqb, g.nkb, status);
+                                                       g.nqb, g.nkb, status, wait_limit(g));
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -33,7 +33,6 @@ namespace sla {
 
 namespace {
 
-constexpr long long kTimeout = 1ll << 31;
 constexpr int kLStages = 3;
 constexpr uint32_t kLPart = 128 * 128;         // 128 rows x 32 fp32 (128 B)
 constexpr uint32_t kLStage = 4 * kLPart;       // A hi, A lo, B hi, B lo
@@ -52,7 +51,7 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
     const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
     const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
     float* __restrict__ logits, int nqb, int nkb, int kchunks, int tiles_m, int tiles_n, int ntiles,
-    float scale, int32_t* status) {
+    float scale, int32_t* status, long long timeout, int debug_skip) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const uint32_t sb = smem_u32(base);
@@ -89,8 +88,9 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
       coords(t, m0, n0, bh);
       for (int ks = 0; ks < kchunks && ok; ++ks, ++g) {
         const int s = g % kLStages;
-        if (g >= kLStages) ok = wait_bounded(b_empty(s), ((g / kLStages) & 1) ^ 1, status, kTimeout);
+        if (g >= kLStages) ok = wait_bounded(b_empty(s), ((g / kLStages) & 1) ^ 1, status, timeout);
         if (!ok) break;
+        if (debug_skip && blockIdx.x == 0 && g == 0) continue;  // test aid: this chunk never arrives
         const uint32_t st = sb + s * kLStage;
         mbar_expect_tx(b_full(s), kLStage);
         tma_load_3d(st, &tmQh, ks * 32, m0, bh, b_full(s));
@@ -106,10 +106,10 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
       const int a = it & 1;
       // the epilogue has drained this accumulator (tile it - 2)
-      if (it >= 2) ok = wait_bounded(b_acc_empty(a), ((it >> 1) & 1) ^ 1, status, kTimeout);
+      if (it >= 2) ok = wait_bounded(b_acc_empty(a), ((it >> 1) & 1) ^ 1, status, timeout);
       for (int ks = 0; ks < kchunks && ok; ++ks, ++g) {
         const int s = g % kLStages;
-        ok = wait_bounded(b_full(s), (g / kLStages) & 1, status, kTimeout);
+        ok = wait_bounded(b_full(s), (g / kLStages) & 1, status, timeout);
         if (!ok) break;
         tc_fence_after();
         const uint32_t acc = tmem + 128 * a;
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
       const int a = it & 1;
       int m0, n0, bh;
       coords(t, m0, n0, bh);
-      ok = __all_sync(0xffffffffu, wait_bounded(b_acc_full(a), (it >> 1) & 1, status, kTimeout));
+      ok = __all_sync(0xffffffffu, wait_bounded(b_acc_full(a), (it >> 1) & 1, status, timeout));
       if (!ok) break;  // (the whole warp: the loop below synchronises it)
       tc_fence_after();
       const int row0 = m0 + quad * 32;
@@ -200,7 +200,8 @@ cudaError_t launch_logits_tc(const float* qhi, const float* qlo, const float* kh
   if (e != cudaSuccess) return e;
   const int grid = std::min(ntiles, sm_count());
   logits_tc_kernel<<<grid, 192, kLSmem, s>>>(mQh, mQl, mKh, mKl, logits, g.nqb, g.nkb, g.d / 32, tiles_m,
-                                             tiles_n, ntiles, g.scale, status);
+                                             tiles_n, ntiles, g.scale, status, wait_limit(g),
+                                             debug_withhold(g, SLA_WITHHOLD_LOGITS) ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -283,9 +283,6 @@ struct ClassifyArgs {
   int32_t* tie_count;
 };
 
-__device__ __forceinline__ uint64_t to_fixed(uint32_t pbits) {
-  return __double2ull_rz(static_cast<double>(__uint_as_float(pbits)) * kFixedOne);
-}
 
 template <int CT>
 struct SelShared {

@@ -38,7 +38,12 @@ sla_status make_geom(const sla_params* p, Geom* g) {
     return SLA_ERR_INVALID_ARG;
   if (p->mask_mode == SLA_MASK_CDF && !(p->thr >= 0.0 && p->thr < 1.0)) return SLA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0f) || !isfinite(p->scale)) return SLA_ERR_INVALID_ARG;
-  if (p->flags & ~(SLA_FLAG_SIMT | SLA_FLAG_DEBUG_TIMEOUT)) return SLA_ERR_INVALID_ARG;
+  if (p->flags & ~(SLA_FLAG_SIMT | SLA_FLAG_DEBUG_TIMEOUT | SLA_DEBUG_WITHHOLD(0xF)))
+    return SLA_ERR_INVALID_ARG;
+  if ((p->flags & SLA_DEBUG_WITHHOLD(0xF)) &&
+      (!(p->flags & SLA_FLAG_DEBUG_TIMEOUT) ||
+       ((p->flags >> 8) & 0xF) > SLA_WITHHOLD_BWD_DKDV))
+    return SLA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if ((p->block_q != 64 && p->block_q != 128) || (p->block_k != 64 && p->block_k != 128))
     return SLA_ERR_UNSUPPORTED;
@@ -299,6 +304,7 @@ sla_status sla_linear_combine(const sla_params* p, const void* q, const void* k,
   const FwdWs w = fwd_ws(g);
   if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
   if (!has_linear_branch(g)) {
     SLA_CUDA(sla::launch_combine_copy(o_s, out, o_lin, g, s));
     return SLA_OK;
@@ -513,7 +519,9 @@ sla_status sla_check_device_status(void* ws, void* stream) {
 // none) lives in one file-scope device array of kNoAllocBytes.  Host code
 // only ever sees a host-side stand-in for the array's name, so the device
 // address is looked up once per device, with that device current, by the
-// first call on it, and cached.
+// first call on it, and cached together with the id of the context it
+// belongs to; a later call under another context (after cudaDeviceReset,
+// the module is loaded again and the array may move) looks it up again.
 
 #include <mutex>
 
@@ -522,6 +530,7 @@ constexpr size_t kNoAllocBytes = size_t(16) << 20;  // 16 MiB
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocMaxDevices] = {};
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
@@ -546,11 +555,15 @@ extern "C" sla_status sla_sparse_attention_noalloc(const sla_params* p, const vo
   void* base = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_addr[dev]) {
+    unsigned long long ctx = 0;
+    const bool have_ctx = sla::current_context_id(&ctx);
+    if (!g_noalloc_addr[dev] || (have_ctx && ctx != g_noalloc_ctx[dev])) {
       void* addr = nullptr;
       if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr)
         return SLA_ERR_CUDA;
       g_noalloc_addr[dev] = addr;
+      // (the first call creates the context when there is none yet)
+      g_noalloc_ctx[dev] = sla::current_context_id(&ctx) ? ctx : 0;
     }
     base = g_noalloc_addr[dev];
   }

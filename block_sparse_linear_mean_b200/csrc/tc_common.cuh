@@ -246,33 +246,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two lanes on the FMA pipe, relieving the special-function unit.
-// Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer j in
-// the low mantissa bits of the sum, f = x - j lies in [-1/2, 1/2], 2^f is a
-// cubic (near-minimax in relative error, 7.5e-5, fitted by exp2_poly_fit.py
-// beside this file), and j is added to the exponent field.  x is clamped
-// below at -126 so the exponent stays in range (2^-126 stands in for
-// anything smaller); x must be at most 127.  The error is far below the
-// bf16 rounding the result goes through next.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = add2(x, make_float2(kShift, kShift));
-  const float2 j = add2(t, make_float2(-kShift, -kShift));
-  const float2 f = add2(x, make_float2(-j.x, -j.y));
-  float2 p = fma2(f, make_float2(0.0551716648042202f, 0.0551716648042202f),
-                  make_float2(0.2426111251115799f, 0.2426111251115799f));
-  p = fma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = fma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  // j sits in the low bits of t: p + t * 2^23 (mod 2^32) adds j to p's
-  // exponent in one multiply-add
-  uint32_t rx, ry;
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(p.x)));
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(p.y)));
-  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
-}
-
 // A descriptor advanced by `bytes` (a multiple of 16): the start address
 // field holds address / 16 in its low 14 bits, and shared addresses stay
 // below 256 KB, so the add never carries out of the field.  Building each

@@ -22,6 +22,28 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool tma_available() { return encode_fn() != nullptr; }
 
+// Unique id of the calling thread's current CUDA context (never reused in a
+// process, unlike the context handle), through the driver entry points.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    looked_up = true;
+  }
+  CUcontext c = nullptr;
+  if (!get_ctx || !get_id || get_ctx(&c) != CUDA_SUCCESS || !c) return false;
+  return get_id(c, id) == CUDA_SUCCESS;
+}
+
 // SMs of the current device (persistent kernels launch one CTA per SM, or a
 // fixed number per SM); 148 if the query fails.
 int sm_count() {

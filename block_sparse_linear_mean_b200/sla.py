@@ -33,6 +33,14 @@ SLA_MASK_TOPK, SLA_MASK_CDF = 0, 1
 SLA_OP_MASK, SLA_OP_FORWARD, SLA_OP_BACKWARD = 0, 1, 2
 SLA_FLAG_SIMT = 1
 SLA_FLAG_DEBUG_TIMEOUT = 2
+# SLA_DEBUG_WITHHOLD(kernel): which tensor-core kernel withholds a load under
+# SLA_FLAG_DEBUG_TIMEOUT
+(SLA_WITHHOLD_ATTENTION, SLA_WITHHOLD_LOGITS, SLA_WITHHOLD_SUMMARIES, SLA_WITHHOLD_GATHER,
+ SLA_WITHHOLD_BWD_DQ, SLA_WITHHOLD_BWD_DKDV) = range(6)
+
+
+def SLA_DEBUG_WITHHOLD(kernel: int) -> int:
+    return kernel << 8
 # block labels in the int8 mask
 CRITICAL, MARGINAL, NEGLIGIBLE = 2, 1, 0
 
@@ -398,6 +406,35 @@ def forward(p: sla_params, q, k, v, proj, rows: BlockLists, save_for_backward=Fa
                                       lse.data_ptr(), _ptr(o_s), _ptr(o_lin),
                                       ws.data_ptr(), ws.numel(), _stream()))
     return dict(out=out, lse=lse, o_s=o_s, o_lin=o_lin, ws=ws)
+
+
+def sparse_attention(p: sla_params, q, k, v, rows: BlockLists,
+                     ws: Optional[torch.Tensor] = None) -> dict:
+    """Critical part alone (``sla_sparse_attention``): O_s and LSE in fp32."""
+    dev = q.device
+    o_s = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(p, SLA_OP_FORWARD, dev)
+    _check("sla_sparse_attention", sla_sparse_attention(
+        p, q.data_ptr(), k.data_ptr(), v.data_ptr(), rows.c(), o_s.data_ptr(), lse.data_ptr(),
+        ws.data_ptr(), ws.numel(), _stream()))
+    return dict(o_s=o_s, lse=lse, ws=ws)
+
+
+def linear_combine(p: sla_params, q, k, v, proj, rows: BlockLists, o_s: torch.Tensor,
+                   save_o_lin=False, ws: Optional[torch.Tensor] = None) -> dict:
+    """Marginal part and combine (``sla_linear_combine``): out = o_s +
+    O_lin @ proj in the input dtype, O_lin optionally in fp32."""
+    dev = q.device
+    out = torch.empty_like(q)
+    o_lin = torch.empty(q.shape, dtype=torch.float32, device=dev) if save_o_lin else None
+    if ws is None:
+        ws = workspace(p, SLA_OP_FORWARD, dev)
+    _check("sla_linear_combine", sla_linear_combine(
+        p, q.data_ptr(), k.data_ptr(), v.data_ptr(), proj.data_ptr(), rows.c(), o_s.data_ptr(),
+        out.data_ptr(), _ptr(o_lin), ws.data_ptr(), ws.numel(), _stream()))
+    return dict(out=out, o_lin=o_lin, ws=ws)
 
 
 def backward(p: sla_params, q, k, v, proj, dout, rows: BlockLists, cols: BlockLists,

@@ -101,11 +101,22 @@ typedef struct {
 /* Force the portable fp32 SIMT kernels even for bf16 inputs, and the fp32
  * FMA pooled logits (testing aid). */
 #define SLA_FLAG_SIMT 1
-/* Testing aid for the failure path: the tensor-core attention kernel's first
- * CTA withholds one K/V tile load and every bounded device-side wait gives up
- * after ~1e7 cycles instead of ~2e9, so the call ends with SLA_ERR_TIMEOUT in
- * the status word (read by sla_check_device_status) instead of hanging. */
+/* Testing aid for the failure path: every bounded device-side wait gives up
+ * after ~1.7e7 cycles instead of ~2.1e9, and the first CTA of one tensor-core
+ * kernel withholds one tile load, so the call ends with SLA_ERR_TIMEOUT in the
+ * status word (read by sla_check_device_status) instead of hanging.  The
+ * kernel is chosen with SLA_DEBUG_WITHHOLD(kernel) in the same flags word
+ * (default: the attention forward); the flag makes no kernel fault. */
 #define SLA_FLAG_DEBUG_TIMEOUT 2
+#define SLA_DEBUG_WITHHOLD(kernel) ((kernel) << 8)
+typedef enum {
+  SLA_WITHHOLD_ATTENTION = 0,  /* sla_forward / sla_attention_combine / sla_sparse_attention */
+  SLA_WITHHOLD_LOGITS = 1,     /* sla_build_mask: pooled logits on the tensor cores         */
+  SLA_WITHHOLD_SUMMARIES = 2,  /* sla_forward(_prepare): key-block summaries H_j            */
+  SLA_WITHHOLD_GATHER = 3,     /* sla_forward(_prepare): marginal sums H^M_i                */
+  SLA_WITHHOLD_BWD_DQ = 4,     /* sla_backward: dQ kernel                                   */
+  SLA_WITHHOLD_BWD_DKDV = 5    /* sla_backward: dK, dV kernel                               */
+} sla_withhold_kernel;
 
 /* Compressed block lists.  Row lists (CSR): for each of the B*H*Nqb query
  * blocks r, crit_cnt[r] critical key-block indices in ascending order at
@@ -232,8 +243,9 @@ SLA_API sla_status sla_sparse_attention(const sla_params* p, const void* q, cons
  * B*H*ceil(N/128)*Nkb*4 bytes; the 1.3B-DiT shape needs 6.3 MB, the
  * 14B-DiT and long-clip shapes are refused).
  * The first call on each device looks up the array's device address (a
- * one-time set-up per device); make that first call before any stream
- * capture.  All calls share the array and it keeps the last call's
+ * one-time set-up per device, repeated only when the device's context has
+ * changed, e.g. after cudaDeviceReset); make that first call before any
+ * stream capture.  All calls share the array and it keeps the last call's
  * contents: calls that may overlap on the GPU (other streams, other host
  * threads) race with each other and must be serialised by the caller. */
 SLA_API sla_status sla_sparse_attention_noalloc(const sla_params* p, const void* q,

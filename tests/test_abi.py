@@ -96,9 +96,19 @@ def good_params(**kw):
     ("frac_marg", 0.96, sla.SLA_ERR_INVALID_ARG),   # 0.05 + 0.96 > 1
     ("scale", float("nan"), sla.SLA_ERR_INVALID_ARG),
     ("flags", 8, sla.SLA_ERR_INVALID_ARG),
+    # a withheld-load selector without the debug flag, or past the last kernel
+    ("flags", sla.SLA_DEBUG_WITHHOLD(sla.SLA_WITHHOLD_GATHER), sla.SLA_ERR_INVALID_ARG),
+    ("flags", sla.SLA_FLAG_DEBUG_TIMEOUT | sla.SLA_DEBUG_WITHHOLD(6), sla.SLA_ERR_INVALID_ARG),
+    ("flags", 1 << 12, sla.SLA_ERR_INVALID_ARG),
 ])
 def test_validation_rejects(lib, field, value, expect):
     assert sla.sla_validate(good_params(**{field: value})) == expect
+
+
+def test_validation_accepts_every_withheld_load_selector(lib):
+    for kernel in range(sla.SLA_WITHHOLD_BWD_DKDV + 1):
+        flags = sla.SLA_FLAG_DEBUG_TIMEOUT | sla.SLA_DEBUG_WITHHOLD(kernel)
+        assert sla.sla_validate(good_params(flags=flags)) == sla.SLA_OK
 
 
 def test_validation_cdf_threshold_range(lib):
