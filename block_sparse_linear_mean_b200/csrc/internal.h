@@ -64,6 +64,17 @@ cudaError_t launch_logits_tc(const float* qhi, const float* qlo, const float* kh
 cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
                             const sla_block_lists& rows, float* scores,
                             int32_t* tie_count, cudaStream_t s, bool from_prob = false);
+// one warp per row: logits (or row-softmaxed scores, from_prob) of `nrows`
+// rows -> mask, row lists, optional scores; near-ties added to *tie_count
+// (mask_select.cu)
+cudaError_t launch_select_rows(const float* in, int nrows, const Geom& g, int8_t* mask,
+                               const sla_block_lists& rows, float* scores, int32_t* tie_count,
+                               bool from_prob, cudaStream_t s);
+// 3D-tile token order and the row permutation (tile_order.cu)
+cudaError_t launch_tile_order(int F, int R, int C, int tf, int tr, int tc, int32_t* perm,
+                              cudaStream_t s);
+cudaError_t launch_permute_rows(const void* src, void* dst, const int32_t* perm, i64 rows, int N,
+                                int row_bytes, bool scatter, cudaStream_t s);
 cudaError_t launch_rows_from_mask(const int8_t* mask, const Geom& g,
                                   const sla_block_lists& rows, cudaStream_t s);
 cudaError_t launch_cols_from_mask(const int8_t* mask, const Geom& g,

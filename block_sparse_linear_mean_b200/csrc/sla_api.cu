@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include "internal.h"
 
 namespace sla {
@@ -14,6 +16,11 @@ using sla::Geom;
 namespace {
 
 constexpr size_t kStatusBytes = 256;
+// The pooled logits of the mask step are produced and classified a group of
+// heads at a time through a slab of at most this size, which stays in L2
+// (126 MB) between the two kernels: the whole [B, H, Nqb, Nkb] score matrix
+// never goes to HBM.
+constexpr size_t kSlabBytes = size_t(48) << 20;
 
 size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -87,6 +94,13 @@ bool bwd_tc_attention(const Geom& g) {
 }
 bool bwd_tc_linear(const Geom& g) { return bwd_tc_attention(g) && sla::lin_tc_supported(g); }
 
+// Heads per group of the mask step (the slab holds their logits).
+int mask_group_heads(const Geom& g) {
+  const size_t per_head = sizeof(float) * size_t(g.nqb) * g.nkb;
+  const size_t fit = std::max<size_t>(1, kSlabBytes / per_head);
+  return static_cast<int>(std::min<size_t>(fit, size_t(g.BH)));
+}
+
 MaskWs mask_ws(const Geom& g) {
   MaskWs w;
   size_t off = kStatusBytes;
@@ -97,9 +111,19 @@ MaskWs mask_ws(const Geom& g) {
     w.qlo = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.d);
     w.klo = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nkb * g.d);
   }
-  w.logits = off; off = align_up(off + sizeof(float) * size_t(g.BH) * g.nqb * g.nkb);
+  w.logits = off;
+  off = align_up(off + sizeof(float) * size_t(mask_group_heads(g)) * g.nqb * g.nkb);
   w.total = off;
   return w;
+}
+
+sla_block_lists lists_from_row(const sla_block_lists& l, size_t row, int width) {
+  sla_block_lists r = l;
+  r.crit_cnt += row;
+  r.marg_cnt += row;
+  r.crit_idx += row * width;
+  r.marg_idx += row * width;
+  return r;
 }
 
 FwdWs fwd_ws(const Geom& g) {
@@ -219,17 +243,40 @@ sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
   float* qbar = at<float>(ws, w.qbar);
   float* kbar = at<float>(ws, w.kbar);
   float* logits = at<float>(ws, w.logits);
+  if (tie_count) SLA_CUDA(cudaMemsetAsync(tie_count, 0, sizeof(int32_t), s));
+  const size_t rowcols = size_t(g.nqb) * g.nkb;
   if (sla::logits_tc_supported(g)) {
     float* qlo = at<float>(ws, w.qlo);
     float* klo = at<float>(ws, w.klo);
     SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, qlo, klo, g.BH, g.N, g.d, g.bq, g.bk, s));
-    SLA_CUDA(sla::launch_logits_tc(qbar, qlo, kbar, klo, logits, g, at<int32_t>(ws, 0), s));
+    // logits and selection a group of heads at a time, through the slab
+    const int G = mask_group_heads(g);
+    for (int h0 = 0; h0 < g.BH; h0 += G) {
+      Geom gg = g;
+      gg.BH = std::min(G, g.BH - h0);
+      const size_t qo = size_t(h0) * g.nqb * g.d, ko = size_t(h0) * g.nkb * g.d;
+      SLA_CUDA(sla::launch_logits_tc(qbar + qo, qlo + qo, kbar + ko, klo + ko, logits, gg,
+                                     at<int32_t>(ws, 0), s));
+      SLA_CUDA(sla::launch_select_rows(logits, gg.BH * g.nqb, g, mask + h0 * rowcols,
+                                       lists_from_row(*rows, size_t(h0) * g.nqb, g.nkb),
+                                       scores ? scores + h0 * rowcols : nullptr, tie_count,
+                                       false, s));
+    }
   } else {
     SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, nullptr, nullptr, g.BH, g.N, g.d, g.bq, g.bk,
                               s));
-    SLA_CUDA(sla::launch_logits(qbar, kbar, logits, g, s));
+    const int G = mask_group_heads(g);
+    for (int h0 = 0; h0 < g.BH; h0 += G) {
+      Geom gg = g;
+      gg.BH = std::min(G, g.BH - h0);
+      SLA_CUDA(sla::launch_logits(qbar + size_t(h0) * g.nqb * g.d, kbar + size_t(h0) * g.nkb * g.d,
+                                  logits, gg, s));
+      SLA_CUDA(sla::launch_select_rows(logits, gg.BH * g.nqb, g, mask + h0 * rowcols,
+                                       lists_from_row(*rows, size_t(h0) * g.nqb, g.nkb),
+                                       scores ? scores + h0 * rowcols : nullptr, tie_count,
+                                       false, s));
+    }
   }
-  SLA_CUDA(sla::launch_classify(logits, g, mask, *rows, scores, tie_count, s));
   if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
   return SLA_OK;
 }
@@ -245,7 +292,8 @@ sla_status sla_classify_scores(const sla_params* p, const float* scores,
       (cols && !lists_ok(cols)) || (tie_count && (reinterpret_cast<uintptr_t>(tie_count) & 3u)))
     return SLA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  SLA_CUDA(sla::launch_classify(scores, g, mask, *rows, nullptr, tie_count, s, true));
+  if (tie_count) SLA_CUDA(cudaMemsetAsync(tie_count, 0, sizeof(int32_t), s));
+  SLA_CUDA(sla::launch_select_rows(scores, g.BH * g.nqb, g, mask, *rows, nullptr, tie_count, true, s));
   if (cols) SLA_CUDA(sla::launch_cols_from_mask(mask, g, *cols, s));
   return SLA_OK;
 }
@@ -497,6 +545,34 @@ sla_status sla_mask_recall(const sla_params* p, const int8_t* mask, const float*
       !aligned16(counts))
     return SLA_ERR_INVALID_ARG;
   SLA_CUDA(sla::launch_mask_recall(mask, importance, g, counts, static_cast<cudaStream_t>(stream)));
+  return SLA_OK;
+}
+
+sla_status sla_tile_order(int32_t F, int32_t R, int32_t C, int32_t tf, int32_t tr, int32_t tc,
+                          int32_t* perm, void* stream) {
+  if (F < 1 || R < 1 || C < 1 || tf < 1 || tr < 1 || tc < 1 || !perm ||
+      (reinterpret_cast<uintptr_t>(perm) & 3u))
+    return SLA_ERR_INVALID_ARG;
+  if (int64_t(F) * R * C >= (int64_t(1) << 31)) return SLA_ERR_UNSUPPORTED;
+  SLA_CUDA(sla::launch_tile_order(F, R, C, std::min(tf, F), std::min(tr, R), std::min(tc, C), perm,
+                                  static_cast<cudaStream_t>(stream)));
+  return SLA_OK;
+}
+
+sla_status sla_permute_tokens(const sla_params* p, const void* src, void* dst, const int32_t* perm,
+                              int32_t elem_bytes, int32_t inverse, void* stream) {
+  Geom g;
+  sla_status st = make_geom(p, &g);
+  if (st != SLA_OK) return st;
+  if (!tensor_ok(src) || !tensor_ok(dst) || !perm || (reinterpret_cast<uintptr_t>(perm) & 3u) ||
+      (elem_bytes != 2 && elem_bytes != 4) || (inverse != 0 && inverse != 1))
+    return SLA_ERR_INVALID_ARG;
+  const int row_bytes = g.d * elem_bytes;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(src), b = reinterpret_cast<uintptr_t>(dst);
+  const uintptr_t bytes = static_cast<uintptr_t>(g.BH) * g.N * row_bytes;
+  if (a < b + bytes && b < a + bytes) return SLA_ERR_INVALID_ARG;  // overlapping
+  SLA_CUDA(sla::launch_permute_rows(src, dst, perm, static_cast<sla::i64>(g.BH) * g.N, g.N, row_bytes,
+                                    inverse != 0, static_cast<cudaStream_t>(stream)));
   return SLA_OK;
 }
 
