@@ -61,9 +61,6 @@ cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
 bool logits_tc_supported(const Geom& g);
 cudaError_t launch_logits_tc(const float* qhi, const float* qlo, const float* khi, const float* klo,
                              float* logits, const Geom& g, int32_t* status, cudaStream_t s);
-cudaError_t launch_classify(const float* logits, const Geom& g, int8_t* mask,
-                            const sla_block_lists& rows, float* scores,
-                            int32_t* tie_count, cudaStream_t s, bool from_prob = false);
 // one warp per row: logits (or row-softmaxed scores, from_prob) of `nrows`
 // rows -> mask, row lists, optional scores; near-ties added to *tie_count
 // (mask_select.cu)

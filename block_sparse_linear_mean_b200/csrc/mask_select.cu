@@ -89,8 +89,8 @@ __device__ __forceinline__ void bin_from_top(const uint32_t* hcnt, int need, int
 // reaches thr (thr > 0); below = the mass of the bins under b, above = the
 // scores in the bins over b.  found = false when the whole row's mass stays
 // under thr.  Lane l walks bins 8l + i.
-__device__ __forceinline__ void bin_from_bottom(const uint32_t* hcnt, const unsigned long long* hmass,
-                                                uint64_t thr, int lane, int& bin,
+__device__ __forceinline__ void bin_from_bottom(const uint32_t* hcnt, const uint32_t* hmass,
+                                                uint32_t thr, int lane, int& bin,
                                                 unsigned long long& below, int& above, bool& found) {
   unsigned long long c[8], local = 0;
   uint32_t n[8], nloc = 0;
@@ -246,7 +246,7 @@ __host__ __device__ __forceinline__ WarpMem warp_mem(int nkb, bool cdf) {
   const size_t nkb4 = (static_cast<size_t>(nkb) + 3) & ~size_t(3);
   WarpMem w;
   size_t off = 0;
-  w.mass = off; off += cdf ? 8 * kBins : 0;
+  w.mass = off; off += cdf ? 4 * kBins : 0;
   w.pb = off; off += 4 * nkb4;
   w.bins = off; off += (nkb4 + 15) & ~size_t(15);
   w.hcnt = off; off += 4 * kBins;
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
   const uint32_t* pb = reinterpret_cast<const uint32_t*>(pf);
   uint32_t* bins = reinterpret_cast<uint32_t*>(wbase + wm.bins);  // one byte per score
   uint32_t* hcnt = reinterpret_cast<uint32_t*>(wbase + wm.hcnt);
-  unsigned long long* hmass = reinterpret_cast<unsigned long long*>(wbase + wm.mass);
+  uint32_t* hmass = reinterpret_cast<uint32_t*>(wbase + wm.mass);  // approximate masses
   uint32_t* cand = reinterpret_cast<uint32_t*>(wbase + wm.cand);
   uint32_t* ctr = reinterpret_cast<uint32_t*>(wbase + wm.ctr);
   const float* lr = in + i64(row) * nkb;
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
   }
   for (int b = lane; b < kBins; b += 32) {
     hcnt[b] = 0u;
-    if (CDF) hmass[b] = 0ull;
+    if (CDF) hmass[b] = 0u;
   }
   if (lane < 4) ctr[lane] = 0u;
   m = warp_max(m);
@@ -345,6 +345,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
     constexpr float kLog2e = 1.4426950408889634f;
     const float ml = m * kLog2e;
     float se = 0.f, emax = 0.f, emin = FLT_MAX;
+#pragma unroll 2
     for (int g = lane; g < G; g += 32) {
       const float4 x = pf4[g];
       float4 e;
@@ -380,6 +381,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
 
   // 3. score patterns, their bins, and the histogram of counts (and
   //    fixed-point masses)
+#pragma unroll 2
   for (int g = lane; g < G; g += 32) {
     const float4 e = pf4[g];
     const float ev[4] = {e.x, e.y, e.z, e.w};
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
       const int j = 4 * g + k;
       if (j < nkb) {
         atomicAdd(&hcnt[b], 1u);
-        if (CDF) atomicAdd(&hmass[b], static_cast<unsigned long long>(to_fixed(v[k])));
+        if (CDF) atomicAdd(&hmass[b], __float2uint_rz(p * 16777216.f));  // 2^-24 units
         if (a.scores) a.scores[off + j] = p;
       }
     }
@@ -521,8 +523,43 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
       int b = 0, ab = 0;
       unsigned long long lo = 0;
       bool found = false;
-      bin_from_bottom(hcnt, hmass, a.thr_fx, lane, b, lo, ab, found);
+      // the bin on the approximate masses, then confirmed (or moved to a
+      // neighbouring non-empty bin) on exact fixed-point sums: the mass under
+      // bin b stays below thr and reaching thr takes bin b
+      bin_from_bottom(hcnt, hmass, static_cast<uint32_t>(a.thr_fx >> 38), lane, b, lo, ab, found);
+      if (!found) b = 255;
+      found = false;
+      for (int it = 0; it <= kBins; ++it) {
+        unsigned long long s_lo = 0, s_b = 0;
+        for (int j = lane; j < nkb; j += 32) {
+          const uint32_t x = pb[j];
+          const int bx = bin_of(x, base, shift);
+          if (bx < b) s_lo += to_fixed(x);
+          else if (bx == b) s_b += to_fixed(x);
+        }
+        s_lo = warp_sum_u64(s_lo);
+        s_b = warp_sum_u64(s_b);
+        if (s_lo >= a.thr_fx) {  // thr is reached below b
+          int nb = b - 1;
+          while (nb > 0 && hcnt[nb] == 0) --nb;
+          b = nb;
+          continue;
+        }
+        if (s_lo + s_b < a.thr_fx) {  // thr is not reached within b
+          int nb = b + 1;
+          while (nb < kBins && hcnt[nb] == 0) ++nb;
+          if (nb >= kBins) break;  // the row's whole mass stays under thr
+          b = nb;
+          continue;
+        }
+        lo = s_lo;
+        found = true;
+        break;
+      }
       if (found) {
+        uint32_t nab = 0;
+        for (int i = lane; i < kBins; i += 32) nab += i > b ? hcnt[i] : 0u;
+        ab = static_cast<int>(__reduce_add_sync(full, nab));
         const bool fit = gather(b, -1);
         const int n = static_cast<int>(min(ctr[0], static_cast<uint32_t>(kCand)));
         uint32_t v;
@@ -638,15 +675,15 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
   // scores straddles a cut): labels are then plain comparisons.
   const bool plain = (!cc.on || cc.fill >= cc.eq) && (!cm.on || cm.fill >= cm.eq);
   const bool want_mb = cc.gap || cm.gap;
-  for (int g0 = 0; plain && g0 < G; g0 += 32) {
-    const int g = g0 + lane;
+  // labels of the group g (four scores) as plain comparisons
+  auto plain_group = [&](int g, bool is_c[4], bool is_m[4], uint32_t& ncl, uint32_t& nml,
+                         uint32_t& lab) {
     uint32_t v[4] = {0u, 0u, 0u, 0u};
     if (g < G) {
       const uint4 v4 = pb4[g];
       v[0] = v4.x; v[1] = v4.y; v[2] = v4.z; v[3] = v4.w;
     }
-    uint32_t ncl = 0, nml = 0, lab = 0;
-    bool is_c[4], is_m[4];
+    ncl = nml = lab = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const bool valid = g < G && 4 * g + k < nkb;
@@ -660,29 +697,41 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
         if (v[k] < cm.v && v[k] > mb_m) mb_m = v[k];
       }
     }
-    const uint32_t pl = ncl | (nml << 16);
-    const uint32_t il = warp_incl_scan(pl, lane);
-    const uint32_t tl = __shfl_sync(full, il, 31);
-    if (g < G) {
-      int pc = nc + static_cast<int>((il - pl) & 0xFFFFu);
-      int pm = nmg + static_cast<int>((il - pl) >> 16);
-      if (pl != 0) {
+  };
+  auto plain_write = [&](int g, const bool is_c[4], const bool is_m[4], uint32_t lab, int pc,
+                         int pm) {
+    if (g >= G) return;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (is_c[k]) a.rows.crit_idx[off + pc++] = 4 * g + k;
-          if (is_m[k]) a.rows.marg_idx[off + pm++] = 4 * g + k;
-        }
-      }
-      if (mask4 && 4 * g + 3 < nkb) {
-        *reinterpret_cast<uint32_t*>(a.mask + off + 4 * g) = lab;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (4 * g + k < nkb) a.mask[off + 4 * g + k] = static_cast<int8_t>((lab >> (8 * k)) & 255u);
-      }
+    for (int k = 0; k < 4; ++k) {
+      if (is_c[k]) a.rows.crit_idx[off + pc++] = 4 * g + k;
+      if (is_m[k]) a.rows.marg_idx[off + pm++] = 4 * g + k;
     }
-    nc += static_cast<int>(tl & 0xFFFFu);
-    nmg += static_cast<int>(tl >> 16);
+    if (mask4 && 4 * g + 3 < nkb) {
+      *reinterpret_cast<uint32_t*>(a.mask + off + 4 * g) = lab;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (4 * g + k < nkb) a.mask[off + 4 * g + k] = static_cast<int8_t>((lab >> (8 * k)) & 255u);
+    }
+  };
+  // two groups per lane and step, list positions from one scan of four
+  // packed 8-bit counts (at most 4 x 32 = 128 each)
+  for (int g0 = 0; plain && g0 < G; g0 += 64) {
+    const int ga = g0 + lane, gb = g0 + 32 + lane;
+    bool ca[4], ma[4], cb[4], mbk[4];
+    uint32_t nca, nma, laba, ncb, nmb, labb;
+    plain_group(ga, ca, ma, nca, nma, laba);
+    plain_group(gb, cb, mbk, ncb, nmb, labb);
+    const uint32_t pk = nca | (nma << 8) | (ncb << 16) | (nmb << 24);
+    const uint32_t inc = warp_incl_scan(pk, lane);
+    const uint32_t ex = inc - pk;
+    const uint32_t tot = __shfl_sync(full, inc, 31);
+    const int ta_c = static_cast<int>(tot & 255u), ta_m = static_cast<int>((tot >> 8) & 255u);
+    plain_write(ga, ca, ma, laba, nc + static_cast<int>(ex & 255u), nmg + static_cast<int>((ex >> 8) & 255u));
+    plain_write(gb, cb, mbk, labb, nc + ta_c + static_cast<int>((ex >> 16) & 255u),
+                nmg + ta_m + static_cast<int>(ex >> 24));
+    nc += ta_c + static_cast<int>((tot >> 16) & 255u);
+    nmg += ta_m + static_cast<int>(tot >> 24);
   }
   for (int g0 = 0; !plain && g0 < G; g0 += 32) {
     const int g = g0 + lane;

@@ -309,6 +309,33 @@ SLA_API sla_status sla_block_importance(const sla_params* p, const void* q, cons
 SLA_API sla_status sla_mask_recall(const sla_params* p, const int8_t* mask,
                                    const float* importance, int32_t* counts, void* stream);
 
+/* Token order of 3D tiles (Veda article, sections "Что произошло" / what
+ * happened and "Контекст" / context: attention is selected over tiles of
+ * tokens, with tile shapes fitted per head and layer).  For a latent grid of
+ * F frames x R rows x C columns in raster order (token t = (f R + r) C + c),
+ * tiles of tf x tr x tc tokens are taken in raster order over the tile grid
+ * (tiles at the far edges are partial) and tokens in raster order inside
+ * each tile, so that a block of consecutive tokens covers a compact box.
+ *   perm   [F*R*C] int32 out (device): perm[n] = raster index of the n-th
+ *          token in tile order
+ * All sizes >= 1 and F*R*C < 2^31; asynchronous on `stream`. */
+SLA_API sla_status sla_tile_order(int32_t F, int32_t R, int32_t C, int32_t tf, int32_t tr,
+                                  int32_t tc, int32_t* perm, void* stream);
+
+/* Moves a token tensor [B, H, N, d] (p's B, H, N, d) into or out of another
+ * token order:
+ *   inverse = 0:  dst[b, h, n, :] = src[b, h, perm[n], :]   (into the order)
+ *   inverse = 1:  dst[b, h, perm[n], :] = src[b, h, n, :]   (back to raster)
+ *   perm        [N] int32 (device), a permutation of 0..N-1 (e.g. from
+ *               sla_tile_order); not checked on the device
+ *   elem_bytes  2 (bf16) or 4 (fp32: the gradients, O_s, O_lin)
+ * src and dst must not overlap.  Running mask, forward and backward on the
+ * permuted q, k, v (and dout) and moving out, dq, dk, dv back gives the
+ * hybrid attention of the tiled blocks in raster order.  Asynchronous. */
+SLA_API sla_status sla_permute_tokens(const sla_params* p, const void* src, void* dst,
+                                      const int32_t* perm, int32_t elem_bytes, int32_t inverse,
+                                      void* stream);
+
 /* Synchronises `stream` and returns the status word the last call on `ws`
  * left (SLA_OK, or SLA_ERR_TIMEOUT when a bounded device-side wait gave up),
  * or SLA_ERR_CUDA when a CUDA error is pending. */
