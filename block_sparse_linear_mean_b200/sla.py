@@ -53,6 +53,7 @@ EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate",
            "sla_linear_combine",
            "sla_backward", "sla_forward_uses_tensor_cores",
            "sla_block_importance", "sla_mask_recall",
+           "sla_tile_order", "sla_permute_tokens",
            "sla_check_device_status")
 
 
@@ -131,6 +132,11 @@ def lib():
         L.sla_block_importance.argtypes = [P(sla_params), VP, VP, VP, VP]
         L.sla_mask_recall.restype = ctypes.c_int
         L.sla_mask_recall.argtypes = [P(sla_params), VP, VP, VP, VP]
+        I32 = ctypes.c_int32
+        L.sla_tile_order.restype = ctypes.c_int
+        L.sla_tile_order.argtypes = [I32, I32, I32, I32, I32, I32, VP, VP]
+        L.sla_permute_tokens.restype = ctypes.c_int
+        L.sla_permute_tokens.argtypes = [P(sla_params), VP, VP, VP, I32, I32, VP]
         L.sla_check_device_status.restype = ctypes.c_int
         L.sla_check_device_status.argtypes = [VP, VP]
         _lib = L
@@ -230,6 +236,14 @@ def sla_block_importance(p, q, k, importance, stream) -> int:
 
 def sla_mask_recall(p, mask, importance, counts, stream) -> int:
     return lib().sla_mask_recall(ctypes.byref(p), mask, importance, counts, stream)
+
+
+def sla_tile_order(F, R, C, tf, tr, tc, perm, stream) -> int:
+    return lib().sla_tile_order(F, R, C, tf, tr, tc, perm, stream)
+
+
+def sla_permute_tokens(p, src, dst, perm, elem_bytes, inverse, stream) -> int:
+    return lib().sla_permute_tokens(ctypes.byref(p), src, dst, perm, elem_bytes, inverse, stream)
 
 
 def sla_check_device_status(ws, stream) -> int:
@@ -452,6 +466,24 @@ def backward(p: sla_params, q, k, v, proj, dout, rows: BlockLists, cols: BlockLi
                                         dk.data_ptr(), dv.data_ptr(), dproj.data_ptr(),
                                         ws.data_ptr(), ws.numel(), _stream()))
     return dict(dq=dq, dk=dk, dv=dv, dproj=dproj, ws=ws)
+
+
+def tile_order(grid, tile, device) -> torch.Tensor:
+    """``perm [F*R*C]`` int32 on ``device``: perm[n] = raster index of the
+    n-th token when the (F, R, C) grid is walked in (tf, tr, tc) tiles."""
+    F, R, C = grid
+    perm = torch.empty(F * R * C, dtype=torch.int32, device=device)
+    _check("sla_tile_order", sla_tile_order(F, R, C, *tile, perm.data_ptr(), _stream()))
+    return perm
+
+
+def permute_tokens(p: sla_params, x: torch.Tensor, perm: torch.Tensor, inverse=False) -> torch.Tensor:
+    """``x [B,H,N,d]`` (bf16 or fp32) moved into the order ``perm``
+    (``out[..., n, :] = x[..., perm[n], :]``), or back with ``inverse``."""
+    out = torch.empty_like(x)
+    _check("sla_permute_tokens", sla_permute_tokens(p, x.data_ptr(), out.data_ptr(), perm.data_ptr(),
+                                                    x.element_size(), 1 if inverse else 0, _stream()))
+    return out
 
 
 def check_device_status(ws: torch.Tensor) -> int:

@@ -171,6 +171,26 @@ def test_mask_quality_entry_points_validate_on_the_host(lib):
     assert sla.sla_mask_recall(bad, 16, 16, 16, None) == sla.SLA_ERR_UNSUPPORTED
 
 
+def test_tile_order_entry_points_validate_on_the_host(lib):
+    # sizes and pointers are checked before anything is enqueued (the
+    # addresses below are never dereferenced)
+    assert sla.sla_tile_order(0, 4, 4, 1, 1, 1, 16, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_tile_order(2, 4, 4, 1, 0, 1, 16, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_tile_order(2, 4, 4, 1, 1, 1, None, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_tile_order(2, 4, 4, 1, 1, 1, 18, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_tile_order(1 << 11, 1 << 10, 1 << 10, 1, 1, 1, 16,
+                              None) == sla.SLA_ERR_UNSUPPORTED
+    p = good_params()
+    big = 1 << 40
+    assert sla.sla_permute_tokens(p, 16, big, 16, 3, 0, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_permute_tokens(p, 16, big, 16, 2, 2, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_permute_tokens(p, 24, big, 16, 2, 0, None) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_permute_tokens(p, 16, big, 18, 2, 0, None) == sla.SLA_ERR_INVALID_ARG
+    # overlapping source and destination
+    assert sla.sla_permute_tokens(p, 1 << 20, (1 << 20) + 4096, 16, 2, 0,
+                                  None) == sla.SLA_ERR_INVALID_ARG
+
+
 def test_workspace_too_small_rejected(lib):
     p = good_params()
     lists = sla.sla_block_lists(16, 16, 16, 16)
