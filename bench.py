@@ -63,9 +63,18 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-range", action="store_true",
+                    help="time only --workload (by default a single-GPU run of the 32k "
+                         "workload also times the 75.6k and 245k workloads)")
+    ap.add_argument("--clock-csv", default=None,
+                    help="also write the raw clock samples of the timed region to this CSV "
+                         "(rank r writes <path>.r when several ranks run)")
     ap.add_argument("--mask-quality", action="store_true",
                     help="instead of the timed step: recall of the workload's mask against "
                          "the dense attention max-pooled over tiles (one GPU; dense work)")
+    ap.add_argument("--tile", default=None,
+                    help="with --mask-quality: also measure blocks of tokens taken in 3D tiles "
+                         "of this shape, e.g. 1,8,8 (frames, rows, columns)")
     return ap.parse_args()
 
 
@@ -79,17 +88,28 @@ def run_mask_quality(args):
     wl = synth.WORKLOADS[args.workload]
     x = synth.make_inputs(wl, seed=0, device=dev)
     p = sla.params_for(wl)
-    m = sla.build_mask(p, x.q, x.k)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    imp = sla.block_importance(p, x.q, x.k)
-    e1.record()
-    rec = sla.mask_recall(p, m["mask"], imp)
-    return {"workload": wl.name, "config": wl.description,
-            "mask_quality": {"reference": "dense attention max-pooled over (query block, key block) "
-                                          "tiles; per row as many reference blocks as the mask keeps",
-                             **{k: (round(v, 4) if isinstance(v, float) else v) for k, v in rec.items()},
-                             "importance_ms": round(e0.elapsed_time(e1), 2)}}
+
+    def measure_recall(q, k):
+        m = sla.build_mask(p, q, k)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        imp = sla.block_importance(p, q, k)
+        e1.record()
+        rec = sla.mask_recall(p, m["mask"], imp)
+        return {**{k: (round(v, 4) if isinstance(v, float) else v) for k, v in rec.items()},
+                "importance_ms": round(e0.elapsed_time(e1), 2)}
+
+    res = {"workload": wl.name, "config": wl.description,
+           "mask_quality": {"reference": "dense attention max-pooled over (query block, key block) "
+                                         "tiles; per row as many reference blocks as the mask keeps",
+                            **measure_recall(x.q, x.k)}}
+    if args.tile:
+        tile = tuple(int(v) for v in args.tile.split(","))
+        perm = sla.tile_order(wl.grid, tile, dev)
+        res["mask_quality_tiled"] = {"tile": list(tile),
+                                     **measure_recall(sla.permute_tokens(p, x.q, perm),
+                                                      sla.permute_tokens(p, x.k, perm))}
+    return res
 
 
 def max_over_ranks(ms: float, device) -> float:
@@ -183,18 +203,17 @@ def backward_flops(wl, mask_np):
 class ClockSampler:
     """Samples SM clock and clock-event (throttle) reasons of one GPU every
     20 ms through NVML in a background thread while the timed region runs;
-    the raw samples are written as CSV, one file per rank, beside the other
-    run outputs."""
+    with ``csv_path`` given, the raw samples are also written there as CSV."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
                "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
-    def __init__(self, device_index, period_s=0.02):
+    def __init__(self, device_index, period_s=0.02, csv_path=None):
         self.idx = device_index
         self.period = period_s
         self.samples = []
         self.err = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = csv_path
 
     def _sample_once(self):
         import pynvml as nv
@@ -241,8 +260,10 @@ class ClockSampler:
             self._sample_once()  # one sample at the end of the timed region
             self._stop.set()
             self.thread.join(timeout=5)
+        if not self.path:
+            return
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             with open(self.path, "w") as f:
                 f.write("t,sm_mhz,reasons_mask,power_w\n")
                 for t, sm, rs, pw in self.samples:
@@ -264,14 +285,86 @@ class ClockSampler:
 
 # --------------------------------------------------------------- our arm
 
+# The metric is quoted over 32k-245k tokens: a default single-GPU run also
+# times these workloads, reported as sub-records of the one JSON line.
+RANGE_WORKLOADS = ("nabla_14b", "long_clip")
 
-def run_ours(args, rank, world, local_rank):
+
+def mask_groups(wl):
+    """Head groups of the mask step: the logits of a group go through a slab
+    of at most 48 MB (the library's constant), one logits and one selection
+    launch per group."""
+    nqb, nkb = math.ceil(wl.N / wl.block_q), math.ceil(wl.N / wl.block_k)
+    bh = wl.B * wl.H
+    per_group = max(1, min(bh, (48 << 20) // (4 * nqb * nkb)))
+    return math.ceil(bh / per_group)
+
+
+def launches_per_step(wl, fused, bwd):
+    """Kernels the library launches per step, from the entry points' code
+    (checked against the ncu launch lists)."""
+    # pool (Q and K in one launch), logits + selection per head group | plan
+    # (+ W to bf16, summaries, indicator, gather GEMM) | fused attention (or
+    # attention + combine)
+    n = 1 + 2 * mask_groups(wl) + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
+        + (1 if (not fused and wl.frac_marg > 0) else 0) + (1 if fused else 2)
+    if bwd:
+        lin = wl.frac_marg > 0
+        n += 1  # column lists
+        if fused and wl.d == 128:
+            # Delta | 2 tile plans, dq (+ linear query side), dkdv (+ linear
+            # key side) | (W to bf16, summaries, indicator, gather of H^M,
+            # indicator + gather of dH, dW partials, dW sum)
+            n += 1 + 4 + (8 if lin else 0)
+        else:
+            # Delta and g, dW partials | dq, dkdv (tcgen05: + 2 tile plans) |
+            # (summaries, linear dq, linear dk dv) | dW reduction
+            n += 2 + (4 if fused else 2) + (3 if lin else 0) + 1
+    return n
+
+
+def stage_bytes(wl, mask_np):
+    """Algorithmic HBM bytes per step of the two memory-bound stages.
+
+    mask: read Q and K once; write the int8 mask, the list entries (4 bytes
+    per critical or marginal block) and the per-row counts (and, for the
+    fine-tune step, the column lists).  The pooled means and scores are the
+    implementation's intermediates, not counted.
+    prepare (linear branch on the tensor cores): read K and V once; write the
+    key-block summaries H_j (bf16 d x d) and z_j (fp32 d) once and read them
+    once; write the per-query-block sums H^M_i, z^M_i once."""
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    esz = 2 if wl.dtype == "bf16" else 4
+    nqb, nkb = math.ceil(N / wl.block_q), math.ceil(N / wl.block_k)
+    listed = int(np.count_nonzero(mask_np))
+    mask_b = 2 * B * H * N * d * esz + B * H * nqb * nkb + 4 * listed + 8 * B * H * nqb
+    if wl.backward:
+        mask_b += 4 * listed + 8 * B * H * nkb
+    prep_b = None
+    if wl.frac_marg > 0 and d == 128 and wl.dtype == "bf16":
+        summ = 2 * d * d + 4 * d
+        prep_b = 2 * B * H * N * d * esz + 2 * B * H * nkb * summ + B * H * nqb * summ
+    return mask_b, prep_b
+
+
+def tensor_peak(peaks, peak_src, timed_s):
+    """The bf16 tensor-core denominator: the burst figure for a timed region
+    under a second, the sustained one (measured under the power cap over
+    seconds) for longer regions."""
+    if timed_s < 1.0:
+        return peaks["bf16_tflops"], f"bf16 dense, burst ({peak_src}; timed region {timed_s:.3f} s)"
+    return (peaks["bf16_tflops_sustained"],
+            f"bf16 dense, sustained ({peak_src}; timed region {timed_s:.3f} s)")
+
+
+def measure(wl, args, rank, world, local_rank, steps, warmup, do_e2e, keep_sample=False):
+    """Time `steps` steps of workload `wl` on this rank's GPU (after
+    `warmup` untimed ones) and return the measurement record."""
     from block_sparse_linear_mean_b200 import sla
     import torch.distributed as dist
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = synth.WORKLOADS[args.workload]
     bwd = wl.backward
     x = synth.make_inputs(wl, seed=rank, device=dev, with_dout=bwd)
     p = sla.params_for(wl)
@@ -295,6 +388,7 @@ def run_ours(args, rank, world, local_rank):
         dq, dk, dv = (torch.empty(x.q.shape, **f32) for _ in range(3))
         dproj = torch.empty(x.proj.shape, **f32)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    ties = torch.zeros(4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
@@ -302,9 +396,9 @@ def run_ours(args, rank, world, local_rank):
         if st != sla.SLA_OK:
             raise sla.SlaError(name, st)
 
-    def stage_mask(q, k):
+    def stage_mask(q, k, tie_ptr=None):
         chk("sla_build_mask", sla.sla_build_mask(p, q.data_ptr(), k.data_ptr(), mask.data_ptr(),
-                                                 rc, cc, None, None, ws_m.data_ptr(),
+                                                 rc, cc, None, tie_ptr, ws_m.data_ptr(),
                                                  ws_m.numel(), sp))
 
     def stage_prepare(k, v):
@@ -326,33 +420,17 @@ def run_ours(args, rank, world, local_rank):
             gk.data_ptr(), gv.data_ptr(), gw.data_ptr(), ws_b.data_ptr(), ws_b.numel(), sp))
 
     fused = sla.sla_forward_uses_tensor_cores(p) == 1 and (wl.frac_marg == 0 or wl.d == 128)
-    # kernels per step: pool (Q and K in one launch), logits, classify | plan
-    # (+ W to bf16, summaries, indicator, gather GEMM) | fused attention (or
-    # attention + combine)
-    launches_per_step = 3 + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
-        + (1 if (not fused and wl.frac_marg > 0) else 0) + (1 if fused else 2)
-    if bwd:
-        lin = wl.frac_marg > 0
-        launches_per_step += 1  # column lists
-        if fused and wl.d == 128:
-            # Delta | 2 tile plans, dq (+ linear query side), dkdv (+ linear
-            # key side) | (W to bf16, summaries, indicator, gather of H^M,
-            # indicator + gather of dH, dW partials, dW sum)
-            launches_per_step += 1 + 4 + (8 if lin else 0)
-        else:
-            # Delta and g, dW partials | dq, dkdv (tcgen05: + 2 tile plans) |
-            # (summaries, linear dq, linear dk dv) | dW reduction
-            launches_per_step += 2 + (4 if fused else 2) + (3 if lin else 0) + 1
-
+    n_launch = launches_per_step(wl, fused, bwd)
 
     # warm-up (also fixes the mask used to count the algorithmic work)
-    for _ in range(max(args.warmup, 0)):
+    for _ in range(max(warmup, 0)):
         stage_mask(x.q, x.k)
         stage_prepare(x.k, x.v)
         stage_combine(x.q, x.k, x.v, out)
         if bwd:
             stage_backward(x.q, x.k, x.v, x.dout)
     torch.cuda.synchronize(dev)
+    assert sla.check_device_status(ws_m) == sla.SLA_OK
     assert sla.check_device_status(ws_f) == sla.SLA_OK
     if bwd:
         assert sla.check_device_status(ws_b) == sla.SLA_OK
@@ -361,12 +439,17 @@ def run_ours(args, rank, world, local_rank):
     bwd_fl = backward_flops(wl, mask_np) if bwd else (0.0, 0.0, 0.0)
     flops += bwd_fl[0]
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clocks:
-        for s in range(args.steps):
+    csv_path = None
+    if args.clock_csv:
+        csv_path = args.clock_csv if world == 1 else f"{args.clock_csv}.{rank}"
+        if wl.name != args.workload:
+            csv_path = f"{csv_path}.{wl.name}"
+    with ClockSampler(local_rank, csv_path=csv_path) as clocks:
+        for s in range(steps):
             flush.zero_()                      # L2 flush, outside the timed events
             e = ev[s]
             e[0].record(stream)
@@ -387,8 +470,13 @@ def run_ours(args, rank, world, local_rank):
     t_comb = [e[2].elapsed_time(e[3]) for e in ev]
     t_bwd = [e[3].elapsed_time(e[4]) for e in ev]
     total_ms = max_over_ranks(sum(e[0].elapsed_time(e[4]) for e in ev), dev)
-    ms_step = total_ms / args.steps
-    value = job_rate(world, flops, args.steps, total_ms)
+    ms_step = total_ms / steps
+    value = job_rate(world, flops, steps, total_ms)
+
+    # the GPU's near-tie count over the whole problem (one untimed call)
+    stage_mask(x.q, x.k, ties.data_ptr())
+    torch.cuda.synchronize(dev)
+    gpu_ties = int(ties[0].item())
 
     # end to end through the C ABI with host buffers: every step copies its
     # inputs (q, k, v, and dO for the fine-tune step) from pinned host memory,
@@ -400,7 +488,7 @@ def run_ours(args, rank, world, local_rank):
     # the first input copy to the last output copy.  Each step's input copy
     # (> L2) replaces the L2 flush.
     e2e = None
-    if not args.no_e2e:
+    if do_e2e:
         ins = (x.q, x.k, x.v, x.dout) if bwd else (x.q, x.k, x.v)
         hosts = [t.cpu().pin_memory() for t in ins]
         nb = 2
@@ -413,13 +501,13 @@ def run_ours(args, rank, world, local_rank):
                    for _ in range(nb)]
         cs, ds = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         mk = lambda: torch.cuda.Event()  # noqa: E731
-        ev_in = [mk() for _ in range(args.steps)]
-        ev_comp = [mk() for _ in range(args.steps)]
-        ev_out = [mk() for _ in range(args.steps)]
+        ev_in = [mk() for _ in range(steps)]
+        ev_comp = [mk() for _ in range(steps)]
+        ev_out = [mk() for _ in range(steps)]
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize(dev)
         t0.record(cs)
-        for s in range(args.steps):
+        for s in range(steps):
             b = s % nb
             with torch.cuda.stream(cs):
                 if s >= nb:
@@ -443,23 +531,23 @@ def run_ours(args, rank, world, local_rank):
                 for h_, d_ in zip(grads_h[b], grads[b]):
                     h_.copy_(d_, non_blocking=True)
                 ev_out[s].record(ds)
-        ds.wait_event(ev_comp[args.steps - 1])
+        ds.wait_event(ev_comp[steps - 1])
         t1.record(ds)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(t0.elapsed_time(t1), dev)
-        e2e = {"value": job_rate(world, flops, args.steps, e2e_ms), "unit": UNIT,
+        e2e = {"value": job_rate(world, flops, steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in ins)),
                "d2h_bytes_per_step": int(out.numel() * out.element_size() +
                                          sum(t.numel() * t.element_size() for t in gsrc)),
-               "ms_per_step": e2e_ms / args.steps,
+               "ms_per_step": e2e_ms / steps,
                "pipelining": "double-buffered, H2D / compute / D2H on three streams"}
 
     peaks, peak_src = load_peaks()
     comb_ms = statistics.mean(t_comb)
     tc = _tc_enabled(p)
     if tc:
-        peak, bound, unit = peaks["bf16_tflops_sustained"], "tensor", "TFLOP/s"
-        peak_note = f"bf16 dense, sustained ({peak_src})"
+        peak, peak_note = tensor_peak(peaks, peak_src, total_ms * 1e-3)
+        bound, unit = "tensor", "TFLOP/s"
     else:
         peak, bound, unit = FP32_SIMT_PEAK_TFLOPS, "alu", "TFLOP/s"
         peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"
@@ -470,15 +558,31 @@ def run_ours(args, rank, world, local_rank):
     achieved = kern_fl / (comb_ms * 1e-3) / 1e12
     roofline = {"bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
                 "unit": unit, "frac": round(achieved / peak, 4),
-                "traffic": TRAFFIC_PER_LAUNCH.get((args.workload, "attn_tc" if tc else "attn_simt")),
+                "traffic": TRAFFIC_PER_LAUNCH.get((wl.name, "attn_tc" if tc else "attn_simt")),
                 "kernel": ("fused tcgen05 attention + linear apply + projection + combine"
                            if fused else "sparse attention forward (SIMT fp32) + combine"),
                 "peak_source": peak_note,
                 "algorithmic": f"{kern_fl:.4g} flops per launch = 4*d*{pairs:.4g} kept critical "
                                f"token pairs + {apply_fl:.4g} linear apply/projection flops"}
+    if tc:
+        roofline["frac_of_sustained"] = round(achieved / peaks["bf16_tflops_sustained"], 4)
+    mask_b, prep_b = stage_bytes(wl, mask_np)
+    hbm = peaks["hbm_gbs"]
+    mask_ms = statistics.mean(t_mask)
+    prep_ms = statistics.mean(t_prep)
+    stages = [{"stage": "mask (pool, score, classify, lists)", "bound": "hbm",
+               "algorithmic_bytes": mask_b, "ms": round(mask_ms, 4),
+               "achieved": round(mask_b / (mask_ms * 1e-3) / 1e9, 1), "peak": hbm,
+               "unit": "GB/s", "frac": round(mask_b / (mask_ms * 1e-3) / 1e9 / hbm, 4)}]
+    if prep_b is not None:
+        stages.append({"stage": "prepare (plan, summaries, marginal sums)", "bound": "hbm",
+                       "algorithmic_bytes": prep_b, "ms": round(prep_ms, 4),
+                       "achieved": round(prep_b / (prep_ms * 1e-3) / 1e9, 1), "peak": hbm,
+                       "unit": "GB/s",
+                       "frac": round(prep_b / (prep_ms * 1e-3) / 1e9 / hbm, 4)})
     res = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (smooth 3D-grid field + noise, seeded)",
         "config": {"workload": wl.description, "name": wl.name, "B": B, "H": H, "N": N, "d": d,
@@ -486,8 +590,8 @@ def run_ours(args, rank, world, local_rank):
                    "frac_crit": wl.frac_crit, "frac_marg": wl.frac_marg, "thr": wl.thr,
                    "parallelism": f"independent problem per GPU x{world}",
                    "l2": "256 MB write flushes L2 between steps, outside the timed events"},
-        "breakdown_ms": {"mask": round(statistics.mean(t_mask), 4),
-                         "prepare (plan + linear summaries + gather)": round(statistics.mean(t_prep), 4),
+        "breakdown_ms": {"mask": round(mask_ms, 4),
+                         "prepare (plan + linear summaries + gather)": round(prep_ms, 4),
                          "attention_combine": round(comb_ms, 4),
                          **({"backward": round(statistics.mean(t_bwd), 4)} if bwd else {})},
         "work": {"effective_flops_per_step": flops, "critical_flops": crit_fl,
@@ -496,11 +600,46 @@ def run_ours(args, rank, world, local_rank):
                     if bwd else {}),
                  "kept_fraction_of_dense_pairs": pairs / (B * H * float(N) * N)},
         "roofline": roofline,
+        "stage_rooflines": stages,
+        "mask_near_tie_rows": gpu_ties,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": n_launch * steps,
         "clocks": clocks.summary(),
     }
-    return res
+    sample = None
+    if keep_sample:
+        # head 0 of batch 0, for the oracle comparison of the CPU-baseline
+        # leg: inputs as drawn, the GPU's mask and the output rows of a few
+        # query blocks spread over the sequence (the last one ragged)
+        blocks = sorted({int(round(i * (nqb - 1) / 7)) for i in range(8)})
+        rows_of = [np.arange(i * wl.block_q, min((i + 1) * wl.block_q, N)) for i in blocks]
+        sample = {"q": x.q[:1, :1].cpu(), "k": x.k[:1, :1].cpu(), "v": x.v[:1, :1].cpu(),
+                  "proj": x.proj.cpu(), "mask": mask_np[:1, :1].copy(), "blocks": blocks,
+                  "out": [out[0, 0, r[0]:r[-1] + 1].float().cpu().numpy() for r in rows_of]}
+    del x, ws_m, ws_f, ws_b, mask, rows, cols, out, o_s, o_lin, lse, flush
+    if bwd:
+        del dq, dk, dv, dproj
+    torch.cuda.empty_cache()
+    return res, sample
+
+
+def run_ours(args, rank, world, local_rank):
+    wl = synth.WORKLOADS[args.workload]
+    res, sample = measure(wl, args, rank, world, local_rank, args.steps, args.warmup,
+                          not args.no_e2e, keep_sample=(rank == 0 and world == 1))
+    if world == 1 and not args.no_range and wl.name == "sla_1p3b":
+        subs = []
+        for name in RANGE_WORKLOADS:
+            r, _ = measure(synth.WORKLOADS[name], args, rank, world, local_rank,
+                           min(args.steps, 10), max(3, min(args.warmup, 3)), False)
+            subs.append({k: r[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup",
+                                           "breakdown_ms", "roofline", "stage_rooflines",
+                                           "mask_near_tie_rows", "gpu_launches", "clocks",
+                                           "work")}
+                        | {"workload": r["config"]["workload"], "name": name,
+                           "N": r["config"]["N"]})
+        res["range"] = subs
+    return res, sample
 
 
 def _tc_enabled(p):
@@ -545,6 +684,41 @@ def cpu_baseline(wl):
             "sample": f"float64 oracle mask + forward on {heads} of {wl.H} heads "
                       f"({secs:.1f} s); value = effective flops of those heads / time",
             "ms_per_call_extrapolated": round(secs / heads * wl.H * 1e3, 1)}
+
+
+def oracle_parity(wl, sample):
+    """The CPU-baseline leg's check of the timed run: the oracle's mask of
+    head 0 (all its rows) against the GPU's, and the oracle's output rows of
+    a few sampled query blocks (with the oracle's own mask row) against the
+    GPU's bf16 output, where the two masks agree on that row."""
+    from oracle import sla_oracle as orc
+    tie_eps = 1e-5
+    ref = orc.build_mask(sample["q"], sample["k"], wl.block_q, wl.block_k, wl.mode,
+                         wl.frac_crit, wl.frac_marg, wl.thr)
+    gm, om = sample["mask"][0, 0], ref["mask"][0, 0]
+    differ = (gm != om).any(axis=-1)
+    ties = ref["margins"][0, 0] <= tie_eps
+    q, k, v = (orc.f64(t[0, 0]) for t in (sample["q"], sample["k"], sample["v"]))
+    w = orc.f64(sample["proj"])
+    errs, over, skipped = [], 0, 0
+    for i, got in zip(sample["blocks"], sample["out"]):
+        if differ[i]:
+            skipped += 1
+            continue
+        o = orc.forward_rows(q, k, v, w, om[i], i, wl.block_q, wl.block_k)["out"]
+        e = np.abs(got.astype(np.float64) - o)
+        errs.append(e)
+        # tolerance: 2e-2 plus the bf16 rounding of the stored output
+        over += int((e > 2e-2 + 2.0 ** -8 * np.abs(o)).sum())
+    e = np.concatenate([x.ravel() for x in errs]) if errs else np.zeros(1)
+    return {"head": 0, "mask_rows": int(gm.shape[0]),
+            "mask_rows_differing": int(differ.sum()),
+            "mask_rows_differing_outside_ties": int((differ & ~ties).sum()),
+            "oracle_tie_rows": int(ties.sum()),
+            "sampled_query_blocks": sample["blocks"], "blocks_skipped_mask_differs": skipped,
+            "out_max_abs_err": float(e.max()), "out_mean_abs_err": float(e.mean()),
+            "out_elements_over_tolerance": over,
+            "tolerance": "max abs 2e-2 (+ bf16 output rounding 2^-8 |ref|), mean abs 2e-3"}
 
 
 def run_reference(args, rank, world):
@@ -596,11 +770,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        res, sample = run_ours(args, rank, world, local_rank)
         if rank == 0:
             wl = synth.WORKLOADS[args.workload]
             if not args.no_cpu_baseline and world == 1:
                 res["cpu_baseline"] = cpu_baseline(wl)
+                res["parity"] = oracle_parity(wl, sample)
             print(json.dumps(res))
     finally:
         if world > 1:
