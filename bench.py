@@ -48,9 +48,10 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernel version (dram__bytes_read.sum +
-# dram__bytes_write.sum; command and figures in profiles/); absent = null.
+# dram__bytes_write.sum, the pipeline's own L2 contents, the timed step of
+# `bench.py --steps 1 --warmup 1`); absent = null.
 TRAFFIC_PER_LAUNCH = {
-    ("sla_1p3b", "attn_tc"): 507_041_280 + 92_068_608,
+    ("sla_1p3b", "attn_tc"): 506_990_336 + 136_226_048,
 }
 
 
@@ -72,6 +73,9 @@ def parse():
     ap.add_argument("--mask-quality", action="store_true",
                     help="instead of the timed step: recall of the workload's mask against "
                          "the dense attention max-pooled over tiles (one GPU; dense work)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="time only the first HEADS heads of the workload (a smaller case "
+                         "for profiler captures; the reported workload says so)")
     ap.add_argument("--tile", default=None,
                     help="with --mask-quality: also measure blocks of tokens taken in 3D tiles "
                          "of this shape, e.g. 1,8,8 (frames, rows, columns)")
@@ -85,7 +89,7 @@ def run_mask_quality(args):
     from block_sparse_linear_mean_b200 import sla
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    wl = synth.WORKLOADS[args.workload]
+    wl = with_heads(synth.WORKLOADS[args.workload], args.heads)
     x = synth.make_inputs(wl, seed=0, device=dev)
     p = sla.params_for(wl)
 
@@ -623,11 +627,19 @@ def measure(wl, args, rank, world, local_rank, steps, warmup, do_e2e, keep_sampl
     return res, sample
 
 
+def with_heads(wl, heads):
+    """The workload restricted to its first `heads` heads (profiling cases)."""
+    if heads is None or heads == wl.H:
+        return wl
+    import dataclasses
+    return dataclasses.replace(wl, H=heads, description=f"{wl.description} [first {heads} heads]")
+
+
 def run_ours(args, rank, world, local_rank):
-    wl = synth.WORKLOADS[args.workload]
+    wl = with_heads(synth.WORKLOADS[args.workload], args.heads)
     res, sample = measure(wl, args, rank, world, local_rank, args.steps, args.warmup,
                           not args.no_e2e, keep_sample=(rank == 0 and world == 1))
-    if world == 1 and not args.no_range and wl.name == "sla_1p3b":
+    if world == 1 and not args.no_range and wl.name == "sla_1p3b" and args.heads is None:
         subs = []
         for name in RANGE_WORKLOADS:
             r, _ = measure(synth.WORKLOADS[name], args, rank, world, local_rank,
