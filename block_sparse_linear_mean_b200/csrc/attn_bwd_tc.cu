@@ -60,6 +60,17 @@ __device__ __forceinline__ Step step_of(uint32_t desc, int e, int N) {
   return st;
 }
 
+// Steps present in a tile's plan.  Every lane of the warp reads a share of
+// the plan words at once: one L2 round trip per 32 words instead of one per
+// word before any work starts.  Called by whole warps.
+template <int BLK>
+__device__ __forceinline__ int plan_steps(const uint32_t* ptiles, int T, int N) {
+  int c = 0;
+  for (int t = static_cast<int>(threadIdx.x % 32); t < T; t += 32)
+    c += 1 + (step_of<BLK>(__ldg(ptiles + t), 1, N).present ? 1 : 0);
+  return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+}
+
 struct BwdShared {
   uint64_t* bars;
   volatile int* abort_flag;
@@ -187,11 +198,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   const int T = tile_cnt[tile];
   const uint32_t* ptiles = tiles + static_cast<i64>(tile) * plan_stride;
   // steps present in the plan (all roles count them the same way)
-  int U = 0;
-  for (int t = 0; t < T; ++t) {
-    const uint32_t desc = ptiles[t];
-    U += 1 + (step_of<BK>(desc, 1, N).present ? 1 : 0);
-  }
+  const int U = plan_steps<BK>(ptiles, T, N);
   // linear branch of the tile's query blocks (A: rows 0-63 or the whole
   // 128-row block; B: rows 64-127 when blocks are 64 rows)
   const bool lin_on = D == 128 && lq.marg_cnt != nullptr;
@@ -261,8 +268,10 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       }
       int u = 0;
       bool ok = true;
+      uint32_t desc_next = T > 0 ? ptiles[0] : 0u;  // (a plan word fetched a tile ahead)
       for (int t = 0; ok && t < T; ++t) {
-        const uint32_t desc = ptiles[t];
+        const uint32_t desc = desc_next;
+        if (t + 1 < T) desc_next = ptiles[t + 1];
         for (int e = 0; ok && e < 2; ++e) {
           const Step st = step_of<BK>(desc, e, N);
           if (!st.present) continue;
@@ -449,8 +458,10 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       if (lane == 0) mbar_arrive(b_qt);
     }
     int u = 0;
+    uint32_t desc_next = T > 0 ? ptiles[0] : 0u;  // (a plan word fetched a tile ahead)
     for (int t = 0; ok && t < T; ++t) {
-      const uint32_t desc = ptiles[t];
+      const uint32_t desc = desc_next;
+      if (t + 1 < T) desc_next = ptiles[t + 1];
       for (int e = 0; e < 2; ++e) {
         const Step st = step_of<BK>(desc, e, N);
         if (!st.present) continue;
@@ -756,8 +767,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   const int bh = tile / nkt, kt = tile % nkt;
   const int T = tile_cnt[tile];
   const uint32_t* ptiles = tiles + static_cast<i64>(tile) * plan_stride;
-  int U = 0;
-  for (int t = 0; t < T; ++t) U += 1 + (step_of<BQ>(ptiles[t], 1, N).present ? 1 : 0);
+  const int U = plan_steps<BQ>(ptiles, T, N);
   // linear branch of the tile's key blocks (A: rows 0-63 or the whole
   // 128-row block; B: rows 64-127 when blocks are 64 rows)
   const int ja = BK == 128 ? kt : 2 * kt;
@@ -817,12 +827,28 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       }
       int u = 0;
       bool ok = true;
+      uint32_t desc_next = T > 0 ? ptiles[0] : 0u;  // (a plan word fetched a tile ahead)
       for (int t = 0; ok && t < T; ++t) {
-        const uint32_t desc = ptiles[t];
+        const uint32_t desc = desc_next;
+        if (t + 1 < T) desc_next = ptiles[t + 1];
         for (int e = 0; e < 2; ++e) {
           const Step st = step_of<BQ>(desc, e, N);
           if (!st.present) continue;
           const int s = u % kBwdStages;
+          // this step's -LSE log2(e) and -Delta, loaded before the wait for
+          // the stage so that their latency hides behind it
+          float na[2], nd[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int q = st.row0 + 32 * j + lane;
+            na[j] = -INFINITY;
+            nd[j] = 0.f;
+            if (q < N) {
+              const float l = lse[static_cast<i64>(bh) * N + q];
+              na[j] = l > -INFINITY ? -l * 1.4426950408889634f : -INFINITY;
+              nd[j] = -delta[static_cast<i64>(bh) * N + q];
+            }
+          }
           bool got = true;
           if (lane == 0 && u >= kBwdStages) got = bwait(sh, b_empty(s), ((u / kBwdStages) & 1) ^ 1);
           if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
@@ -838,15 +864,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           float* nl = reinterpret_cast<float*>(base + offSt + s * kStageBytes + 2 * kHalfBytes);
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const int q = st.row0 + 32 * j + lane;
-            float a = -INFINITY, dd = 0.f;
-            if (q < N) {
-              const float l = lse[static_cast<i64>(bh) * N + q];
-              a = l > -INFINITY ? -l * 1.4426950408889634f : -INFINITY;
-              dd = -delta[static_cast<i64>(bh) * N + q];
-            }
-            nl[32 * j + lane] = a;
-            nl[64 + 32 * j + lane] = dd;
+            nl[32 * j + lane] = na[j];
+            nl[64 + 32 * j + lane] = nd[j];
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(b_full(s));
@@ -969,8 +988,10 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     const float2 c2 = make_float2(scale_log2, scale_log2);
     bool ok = true;
     int u = 0;
+    uint32_t desc_next = T > 0 ? ptiles[0] : 0u;  // (a plan word fetched a tile ahead)
     for (int t = 0; ok && t < T; ++t) {
-      const uint32_t desc = ptiles[t];
+      const uint32_t desc = desc_next;
+      if (t + 1 < T) desc_next = ptiles[t + 1];
       for (int e = 0; e < 2; ++e) {
         const Step st = step_of<BQ>(desc, e, N);
         if (!st.present) continue;
