@@ -21,9 +21,9 @@
 //             3-stage ring
 //   warp 1    TMEM owner and MMA issuer: 4 K-steps of 8 channels x 3
 //             products per chunk into one of two 128-column accumulators
-//   warps 2-5 epilogue: TMEM -> registers -> scale -> a per-warp 32 x 32
-//             transpose in shared memory -> coalesced row stores (any Nkb,
-//             ragged tiles masked)
+//   warps 2-5 epilogue: TMEM -> registers -> scale -> each lane stores its
+//             row's 32 columns with 16-byte stores (the destination is the
+//             L2-resident score slab; any Nkb, ragged tiles masked)
 #include <algorithm>
 
 #include "common.cuh"
@@ -36,9 +36,7 @@ namespace {
 constexpr int kLStages = 3;
 constexpr uint32_t kLPart = 128 * 128;         // 128 rows x 32 fp32 (128 B)
 constexpr uint32_t kLStage = 4 * kLPart;       // A hi, A lo, B hi, B lo
-constexpr uint32_t kLXpose = kLStages * kLStage;
-constexpr uint32_t kLXposeWarp = 32 * 33 * 4;  // padded 32 x 32 fp32
-constexpr uint32_t kLBars = kLXpose + 4 * kLXposeWarp;
+constexpr uint32_t kLBars = kLStages * kLStage;
 constexpr size_t kLSmem = kLBars + 256 + 1024;
 static_assert(kLSmem <= 227 * 1024, "shared memory budget");
 
@@ -128,7 +126,6 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
   } else if (warp >= 2) {
     const int quad = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float* xp = reinterpret_cast<float*>(base + kLXpose + quad * kLXposeWarp);
     int it = 0;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
       const int a = it & 1;
@@ -149,18 +146,25 @@ __global__ void __launch_bounds__(192, 1) logits_tc_kernel(
           __syncwarp();
           if (lane == 0) mbar_arrive(b_acc_empty(a));
         }
-        // lane l holds row row0 + l, columns n0 + c0 .. + 31: transpose so
-        // that each store instruction writes 32 consecutive columns of a row
+        // lane l holds row row0 + l, columns n0 + c0 .. + 31, and stores
+        // them itself: the destination is the score slab, which stays in L2,
+        // so 16-byte stores of one row per lane cost less than a transpose
+        // through shared memory into row-coalesced stores
+        const int row = row0 + lane;
+        const int ncol = min(32, nkb - (n0 + c0));
+        if (row < nqb && ncol > 0) {
+          float* dst = logits + (i64(bh) * nqb + row) * nkb + n0 + c0;
+          if (ncol == 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = v[e] * scale;
-        __syncwarp();
-        const int col = n0 + c0 + lane;
-        if (col < nkb) {
-          float* dst = logits + (i64(bh) * nqb + row0) * nkb + col;
-          const int nr = min(32, nqb - row0);
-          for (int rr = 0; rr < nr; ++rr) dst[i64(rr) * nkb] = xp[rr * 33 + lane];
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + e) =
+                  make_float4(v[e] * scale, v[e + 1] * scale, v[e + 2] * scale, v[e + 3] * scale);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (e < ncol) dst[e] = v[e] * scale;
+          }
         }
-        __syncwarp();
       }
     }
   }
