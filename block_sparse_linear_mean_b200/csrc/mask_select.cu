@@ -188,54 +188,69 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
   return x;
 }
 
+// Bitonic sort of one key per lane across the warp, descending (the largest
+// at lane 0), carrying a payload: 15 compare-exchange steps over shuffles.
+// Blocks of k lanes alternate direction; the last stage (k = 32) runs
+// descending over the whole warp.
+__device__ __forceinline__ void warp_sort_desc(uint32_t& x, unsigned long long& pay, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+      const unsigned long long py = __shfl_xor_sync(0xffffffffu, pay, j);
+      const bool desc = (lane & k) == 0;
+      const bool low = (lane & j) == 0;
+      const bool take_max = low == desc;
+      const bool swap = take_max ? (y > x) : (y < x);
+      if (swap) { x = y; pay = py; }
+    }
+  }
+}
+
 // The candidate at rank need - 1 from the top among n <= 32 candidates held
-// one per lane (`have`): its value, and how many candidates lie above it
-// and equal it.
+// one per lane (`have`; 1 <= need <= n): its value, and how many candidates
+// lie above it and equal it.  Lanes without a candidate sort as 0, below or
+// level with every real one, which leaves the value at rank need - 1 as it is.
 __device__ __forceinline__ void rank_small(uint32_t c, bool have, int need, int lane, uint32_t& v,
                                            int& above, int& eq) {
-  int gt = 0, same = 0;
-#pragma unroll 8
-  for (int k = 0; k < 32; ++k) {
-    const uint32_t ck = __shfl_sync(0xffffffffu, c, k);
-    const bool hk = __shfl_sync(0xffffffffu, have ? 1 : 0, k) != 0;
-    gt += (hk && ck > c) ? 1 : 0;
-    same += (hk && ck == c) ? 1 : 0;
-  }
-  const bool here = have && gt < need && need <= gt + same;
-  const unsigned who = __ballot_sync(0xffffffffu, here);
-  const int src = who ? __ffs(who) - 1 : 0;
-  v = __shfl_sync(0xffffffffu, c, src);
-  above = __shfl_sync(0xffffffffu, gt, src);
-  eq = __shfl_sync(0xffffffffu, same, src);
+  uint32_t key = have ? c : 0u;
+  unsigned long long none = 0;
+  warp_sort_desc(key, none, lane);
+  v = __shfl_sync(0xffffffffu, key, need - 1);
+  above = __popc(__ballot_sync(0xffffffffu, have && c > v));
+  eq = __popc(__ballot_sync(0xffffffffu, have && c == v));
 }
 
 // CDF cut among n <= 32 candidates held one per lane: the candidate v at
 // which lo + (mass of the candidates <= v) first reaches thr, the mass under
 // it (`below`, lo included), and the candidates above and equal to it.
-// found = false if no candidate reaches thr.
+// Sorted descending with their masses, the suffix sums S_L (lane L and
+// every lane after it) decrease with L; v is the key at the last lane with
+// lo + S_L >= thr (a lane of v's group: the group's first lane holds the
+// mass of everything <= v, the lane after the group only what is below v).
 __device__ __forceinline__ void mass_small(uint32_t c, bool have, unsigned long long lo,
                                            uint64_t thr, int lane, uint32_t& v,
                                            unsigned long long& below, int& above, int& eq) {
   const unsigned long long fx = have ? to_fixed(c) : 0ull;
-  unsigned long long lt = 0, le = 0;
-  int gt = 0, same = 0;
-#pragma unroll 8
-  for (int k = 0; k < 32; ++k) {
-    const uint32_t ck = __shfl_sync(0xffffffffu, c, k);
-    const unsigned long long fk = __shfl_sync(0xffffffffu, fx, k);
-    const bool hk = __shfl_sync(0xffffffffu, have ? 1 : 0, k) != 0;
-    if (hk && ck < c) lt += fk;
-    if (hk && ck <= c) le += fk;
-    gt += (hk && ck > c) ? 1 : 0;
-    same += (hk && ck == c) ? 1 : 0;
+  uint32_t key = have ? c : 0u;
+  unsigned long long m = fx;
+  warp_sort_desc(key, m, lane);
+  unsigned long long suf = m;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
   }
-  const bool here = have && lo + lt < thr && thr <= lo + le;
-  const unsigned who = __ballot_sync(0xffffffffu, here);
-  const int src = who ? __ffs(who) - 1 : 0;
-  v = __shfl_sync(0xffffffffu, c, src);
-  below = lo + __shfl_sync(0xffffffffu, lt, src);
-  above = __shfl_sync(0xffffffffu, gt, src);
-  eq = __shfl_sync(0xffffffffu, same, src);
+  const unsigned who = __ballot_sync(0xffffffffu, lo + suf >= thr && m > 0);
+  const int src = who ? 31 - __clz(who) : 0;
+  v = __shfl_sync(0xffffffffu, key, src);
+  unsigned long long under = (have && c < v) ? fx : 0ull;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) under += __shfl_xor_sync(0xffffffffu, under, o);
+  below = lo + under;
+  above = __popc(__ballot_sync(0xffffffffu, have && c > v));
+  eq = __popc(__ballot_sync(0xffffffffu, have && c == v));
 }
 
 // Shared memory of one warp (byte offsets; 16-byte aligned pieces).
