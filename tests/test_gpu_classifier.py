@@ -38,8 +38,9 @@ def _params(nkb, nrows, mode, fc=0.0, fm=0.0, thr=0.0):
 
 
 @pytest.mark.parametrize("kind", ["dups", "zeros", "dyadic", "smooth"])
-# 1-512: one-warp top-k classifier with 16 blocks per lane, 700: 32 per lane,
-# 1920: the one-CTA classifier
+# rows of every length class of the one-warp-per-row kernel (shared memory
+# per warp grows with the row; "dups" rows of 1920 and 2500 blocks overflow
+# the 256 candidate slots and take the exact whole-row search)
 @pytest.mark.parametrize("nkb", [1, 7, 64, 300, 512, 700, 1920, 2500])
 @pytest.mark.parametrize("mode,fc,fm,thr", [("topk", 0.05, 0.10, 0.0), ("topk", 0.5, 0.25, 0.0),
                                             ("cdf", 0.0, 0.0, 0.2), ("cdf", 0.0, 0.1, 0.5),
@@ -66,3 +67,33 @@ def test_classifier_bit_exact_on_crafted_rows(kind, nkb, mode, fc, fm, thr):
     # the GPU's own tie count equals the oracle's on the same values
     if mode == "topk" or kind == "dyadic":
         assert int(got["ties"].item()) == int((margins <= 1e-5).sum())
+
+
+@pytest.mark.parametrize("kind", ["smooth", "dups"])
+@pytest.mark.parametrize("mode,fc,fm,thr", [("topk", 0.03, 0.02, 0.0), ("cdf", 0.0, 0.05, 0.2)])
+def test_classifier_at_the_longest_rows(kind, mode, fc, fm, thr):
+    # rows of 8192 key blocks, the most a mask supports (one warp per CTA,
+    # 68 KB of shared memory); the GPU classifies all 4096 rows, the oracle
+    # a spread of 48 of them
+    nkb, bq = 8192, 128
+    N = nkb * 64
+    nqb = N // bq
+    rng = np.random.default_rng(8192 + len(kind))
+    s32 = _rows(kind, nkb, nqb, rng)
+    wl = synth.Workload(name="cls", B=1, H=1, grid=(1, 1, N), d=64, dtype="f32", block_q=bq,
+                        block_k=64, mode=mode, frac_crit=fc, frac_marg=fm, thr=thr)
+    p = sla.params_for(wl)
+    got = sla.classify_scores(p, torch.from_numpy(s32.reshape(1, 1, nqb, nkb)).cuda())
+    torch.cuda.synchronize()
+    sample = np.linspace(0, nqb - 1, 48).astype(int)
+    mask = got["mask"].cpu().numpy()[0, 0][sample]
+    ref, margins = orc.classify(s32[sample].astype(np.float64), mode, fc, fm, thr)
+    if mode == "topk":
+        np.testing.assert_array_equal(mask, ref)
+    else:
+        diff = (mask != ref).any(axis=-1)
+        assert not (diff & (margins > 1e-12)).any()
+    lists = lists_from_gpu(got["rows"], nqb, nkb)
+    exp = expected_rows(mask[None, None])
+    assert [lists[0][r] for r in sample] == exp[0]
+    assert [lists[1][r] for r in sample] == exp[1]

@@ -220,3 +220,27 @@ def test_bf16_forward_runs_tensor_core_kernel():
     assert sla.sla_forward_uses_tensor_cores(p) == 0        # fp32 mode: SIMT
     p = sla.params_for(synth.WORKLOADS["sla_1p3b"], simt=True)
     assert sla.sla_forward_uses_tensor_cores(p) == 0
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_batch_of_two_matches_oracle(dtype, d):
+    # B = 2: every kernel indexes (batch, head) pairs as one flat index
+    wl = synth.small_case(d=d, grid=(2, 4, 100), H=2, B=2, dtype=dtype, frac_crit=0.2,
+                          frac_marg=0.2)
+    x, t = gpu_inputs(wl, seed=17, with_dout=True)
+    ref = oracle_mask(wl, x)
+    p = sla.params_from(t["q"], wl)
+    m = sla.build_mask(p, t["q"], t["k"], want_scores=True)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(to_np(m["scores"]), ref["scores"], rtol=2e-5, atol=1e-7)
+    compare_masks(m["mask"].cpu().numpy(), ref["mask"], ref["margins"])
+    _, rows, cols = feed_mask(p, ref["mask"])
+    f = sla.forward(p, t["q"], t["k"], t["v"], t["proj"], rows, save_for_backward=True)
+    g = sla.backward(p, t["q"], t["k"], t["v"], t["proj"], t["dout"], rows, cols, f)
+    torch.cuda.synchronize()
+    assert sla.check_device_status(g["ws"]) == sla.SLA_OK
+    o = orc.forward(x.q, x.k, x.v, x.proj, ref["mask"], wl.block_q, wl.block_k)
+    assert_close(to_np(f["out"]), o["out"], dtype, "B2 out", stored_bf16=True)
+    gr = orc.backward(x.q, x.k, x.v, x.proj, ref["mask"], x.dout, wl.block_q, wl.block_k)
+    for key in ("dq", "dk", "dv", "dproj"):
+        assert_close(to_np(g[key]), gr[key], dtype, f"B2 {key}", rel=True)
