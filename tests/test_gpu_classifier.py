@@ -44,7 +44,10 @@ def _params(nkb, nrows, mode, fc=0.0, fm=0.0, thr=0.0):
 @pytest.mark.parametrize("nkb", [1, 7, 64, 300, 512, 700, 1920, 2500])
 @pytest.mark.parametrize("mode,fc,fm,thr", [("topk", 0.05, 0.10, 0.0), ("topk", 0.5, 0.25, 0.0),
                                             ("cdf", 0.0, 0.0, 0.2), ("cdf", 0.0, 0.1, 0.5),
-                                            ("cdf", 0.0, 0.0, 0.0)])
+                                            ("cdf", 0.0, 0.0, 0.0),
+                                            # rows whose fp32 scores sum to just under 1
+                                            # stay under thr: only the top rank is kept
+                                            ("cdf", 0.0, 0.05, 0.99999999)])
 def test_classifier_bit_exact_on_crafted_rows(kind, nkb, mode, fc, fm, thr):
     rng = np.random.default_rng(nkb * 7 + len(kind))
     nrows = nkb  # square: Nqb = Nkb
