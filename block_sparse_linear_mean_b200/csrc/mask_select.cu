@@ -650,9 +650,23 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
         cc.v = pmax;
         cc.fill = 1;
         uint32_t k = 0;
-        for (int j = lane; j < nkb; j += 32) k += pb[j] == pmax ? 1u : 0u;
+        unsigned long long s_all = 0;
+        for (int j = lane; j < nkb; j += 32) {
+          k += pb[j] == pmax ? 1u : 0u;
+          s_all += to_fixed(pb[j]);
+        }
         cc.eq = static_cast<int>(__reduce_add_sync(full, k));
+        s_all = warp_sum_u64(s_all);
         c = 1;
+        if (ties_on && nkb > 1) {
+          // the decisions at the cut: the tail sum of rank 1 against thr,
+          // and rank 1 against the top score (equal, or a relative gap)
+          const double thr = static_cast<double>(a.thr_fx) / kFixedOne;
+          const double t_next = static_cast<double>(s_all - to_fixed(pmax)) / kFixedOne;
+          tie |= fabs(thr - t_next) <= kTieEps;
+          if (cc.eq >= 2) tie = true;
+          else cc.gap = true;
+        }
       }
     }
     const int nm = min(a.n_m, nkb - c);
