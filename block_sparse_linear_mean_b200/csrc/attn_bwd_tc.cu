@@ -524,12 +524,16 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         // rounded values (as the forward forms it)
         float dpart = 0.f, dpart2 = 0.f;
         if (lok) {
+          // all eight pieces read before any is written back (a read after
+          // a store to the same tile would wait for it)
+          uint4 qv[8];
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8) qv[u8] = *reinterpret_cast<const uint4*>(base + offQ + h * 16384 + sw128(r, u8));
 #pragma unroll
           for (int u8 = 0; u8 < 8; ++u8) {
-            uint4* pq = reinterpret_cast<uint4*>(base + offQ + h * 16384 + sw128(r, u8));
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
             if (row < N && nm_r > 0) {
-              val = phi_unit(*pq);
+              val = phi_unit(qv[u8]);
               const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.x));
               const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.y));
               const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.z));
@@ -538,8 +542,10 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
               dpart = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, fmaf(f1.y, za.w, dpart))));
               dpart2 = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, dpart2))));
             }
-            *pq = val;
+            qv[u8] = val;
           }
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8) *reinterpret_cast<uint4*>(base + offQ + h * 16384 + sw128(r, u8)) = qv[u8];
           red[h * 128 + r] = dpart + dpart2;
           __syncwarp();
           if (lane == 0) mbar_arrive(b_den);
@@ -1047,11 +1053,15 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           // phi(K) (rows past N zero): in place for 128-row blocks; for
           // 64-row blocks into the copy of the row's own block, zeros into
           // the other's
+          // (all eight pieces read before any store)
+          uint4 kv[8];
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8) kv[u8] = *reinterpret_cast<const uint4*>(base + offK + h * 16384 + sw128(r, u8));
 #pragma unroll
           for (int u8 = 0; u8 < 8; ++u8) {
             uint4* pk = reinterpret_cast<uint4*>(base + offK + h * 16384 + sw128(r, u8));
             const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-            const uint4 ph = key < N ? phi_unit(*pk) : zero;
+            const uint4 ph = key < N ? phi_unit(kv[u8]) : zero;
             if (BK == 128) {
               *pk = ph;
             } else {

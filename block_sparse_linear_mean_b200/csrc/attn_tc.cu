@@ -350,8 +350,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (clock64() - t0 > timeout_cycles) { give_up(); break; }
         }
       }
-      // linear branch: H^M of the tile's query blocks and W go into the K/V
-      // stages once the last P V product has read them
+      // linear branch: with every K/V load issued (a few tiles before the
+      // end), H^M and z^M of the tile's query blocks -- written by the
+      // gather long before, so in HBM by now -- are prefetched into L2, so
+      // that the epilogue does not wait for HBM
+      if (lin && tv == T) {
+        if (nm_a > 0) {
+          tma_prefetch_2d(&tmHM, 0, (bh * nqb + qa) * 128);
+          tma_prefetch_2d(&tmHM, 64, (bh * nqb + qa) * 128);
+          const float* z = ep.zm + (i64(bh) * nqb + qa) * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) prefetch_l2(z + 32 * i);
+        }
+        if (nm_b > 0) {
+          tma_prefetch_2d(&tmHM, 0, (bh * nqb + qb2) * 128);
+          tma_prefetch_2d(&tmHM, 64, (bh * nqb + qb2) * 128);
+          const float* z = ep.zm + (i64(bh) * nqb + qb2) * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) prefetch_l2(z + 32 * i);
+        }
+      }
+      // H^M of the tile's query blocks and W go into the K/V stages once
+      // the last P V product has read them
       if (lin && tv == T && (T == 0 || wait(b_pv_last, 0))) {
         mbar_expect_tx(b_lin, (nm_a > 0 ? 32768u : 0u) + (nm_b > 0 ? 32768u : 0u) + 32768u);
         if (nm_a > 0) {
@@ -674,12 +694,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float dpart = 0.f, dpart2 = 0.f;
       lin_ok = __all_sync(full, wait(b_q, 0));
       if (lin_ok) {
+        // all eight 16-byte pieces are read before any is written back: a
+        // read after a store to the same region would wait for it, and the
+        // pieces' exponentials would run one after another
+        uint4 qv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) qv[u] = *reinterpret_cast<const uint4*>(base + offQ + h * 16384 + sw128(r, u));
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          uint4* p = reinterpret_cast<uint4*>(base + offQ + h * 16384 + sw128(r, u));
           uint4 val = make_uint4(0u, 0u, 0u, 0u);
           if (row < N && nm_r > 0) {
-            val = phi_unit(*p);
+            val = phi_unit(qv[u]);
             const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.x));
             const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.y));
             const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&val.z));
@@ -688,8 +713,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             dpart = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, fmaf(f1.y, za.w, dpart))));
             dpart2 = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, dpart2))));
           }
-          *p = val;
+          qv[u] = val;
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(base + offQ + h * 16384 + sw128(r, u)) = qv[u];
         dpart += dpart2;
         xch[512 + h * 128 + r] = dpart;
         fence_async_smem();
@@ -707,12 +734,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
         const uint32_t tn = tS(second ? 1 : 0);
         const float dinv = (nm_r > 0 && den > 0.f) ? 1.f / den : 0.f;
+        float vv[64];  // both 32-column chunks in flight before one wait
+        tmem_ld32(tn + lane_off + h * 64, vv);
+        tmem_ld32(tn + lane_off + h * 64 + 32, vv + 32);
+        tmem_wait_ld();
+        reg_fence<64>(vv);
 #pragma unroll
         for (int c = 0; c < 64; c += 32) {
-          float v[32];
-          tmem_ld32(tn + lane_off + h * 64 + c, v);
-          tmem_wait_ld();
-          reg_fence<32>(v);
+          float* v = vv + c;
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = nm_r > 0 ? v[i] * dinv : 0.f;  // TMEM unwritten when no list
           if (ep.o_lin && row < N) {
@@ -740,14 +769,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // final: O / l (+ O_lin W) -> out (bf16) and / or o_s (fp32)
 #pragma unroll
     for (int c = 0; c < DH; c += 32) {
-      float o[32];
+      float o[32], lo[32];
+      // the projection's columns load with the accumulators, one wait for all
+      const bool add_lin = D == 128 && lin_ok && ep.out;
       if (fin && T > 1) {
         float o1[32];
         tmem_ld32(tO(0) + lane_off + h * DH + c, o);
         tmem_ld32(tO(1) + lane_off + h * DH + c, o1);
+        if (add_lin) tmem_ld32(tS(0) + lane_off + h * DH + c, lo);
         tmem_wait_ld();
         reg_fence<32>(o);
         reg_fence<32>(o1);
+        if (add_lin) reg_fence<32>(lo);
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = o[i] * w0 + o1[i] * w1;
       } else if (fin && T > 0) {  // one tile: warpgroup 1 had none
@@ -766,11 +799,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           *reinterpret_cast<float4*>(ep.o_s + orow + c + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
       }
       if (ep.out) {
-        if (D == 128 && lin_ok) {
-          float lo[32];
-          tmem_ld32(tS(0) + lane_off + h * DH + c, lo);
-          tmem_wait_ld();
-          reg_fence<32>(lo);
+        if (add_lin) {
+          if (!(fin && T > 1)) {
+            tmem_ld32(tS(0) + lane_off + h * DH + c, lo);
+            tmem_wait_ld();
+            reg_fence<32>(lo);
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] += lo[i];
         }

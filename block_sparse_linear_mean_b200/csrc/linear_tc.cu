@@ -38,6 +38,34 @@ __device__ __forceinline__ float bf16_at(const uint8_t* tile, int row, int col) 
   return __uint_as_float(static_cast<uint32_t>(bits) << 16);
 }
 
+// phi in place over the first ROWS rows of a bf16 tile of 128 channels kept
+// as two 128-byte-swizzled chunks of 64 channels (`cstride` bytes apart);
+// rows at or past `valid` become zeros.  128 threads, each on ROWS / 8
+// pieces of 16 bytes in batches of up to eight, a batch read before any of
+// it is written back: a read after a store to the same tile would wait for
+// the store, and the pieces' exponentials would run one after another.
+template <int ROWS>
+__device__ __forceinline__ void phi_tile(uint8_t* tile, uint32_t cstride, int valid, int tid) {
+  constexpr int kN = ROWS * 16 / 128, kB = kN < 8 ? kN : 8;  // pieces per thread, per batch
+#pragma unroll
+  for (int b0 = 0; b0 < kN; b0 += kB) {
+    uint4 v[kB];
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int x = tid + 128 * (b0 + i);
+      v[i] = *reinterpret_cast<const uint4*>(tile + ((x >> 3) & 1) * cstride + sw128(x >> 4, x & 7));
+    }
+#pragma unroll
+    for (int i = 0; i < kB; ++i)
+      v[i] = ((tid + 128 * (b0 + i)) >> 4) < valid ? phi_unit(v[i]) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int x = tid + 128 * (b0 + i);
+      *reinterpret_cast<uint4*>(tile + ((x >> 3) & 1) * cstride + sw128(x >> 4, x & 7)) = v[i];
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // 1. Summaries: one CTA (128 threads) per (key block, head).
 //    TMA K_j, V_j -> phi(K) in place (padding rows zeroed) and z_j ->
@@ -78,11 +106,7 @@ __global__ void __launch_bounds__(128) lin_summary_tc_kernel(
   }
   bool ok = __syncthreads_and(wait_bounded(b_tma, 0, status, timeout));
   if (ok) {
-    for (int x = tid; x < BK * 16; x += 128) {
-      const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
-      uint4* p = reinterpret_cast<uint4*>(base + offK + chunk * kChunk + sw128(row, u));
-      *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
-    }
+    phi_tile<BK>(base + offK, kChunk, valid, tid);
     __syncthreads();
     {  // z_j[a] from the rounded phi(K) the MMA uses (four chains, added
        // in a fixed order)
@@ -211,11 +235,7 @@ __global__ void __launch_bounds__(128) lin_summary_persist_kernel(
     }
     ok = __syncthreads_and(wait_bounded(b_tma(b), (k >> 1) & 1, status, timeout));
     if (!ok) break;
-    for (int x = tid; x < BK * 16; x += 128) {
-      const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
-      uint4* p = reinterpret_cast<uint4*>(buf + chunk * kChunk + sw128(row, u));
-      *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
-    }
+    phi_tile<BK>(buf, kChunk, valid, tid);
     __syncthreads();
     {  // z_j[a] from the rounded phi(K) the MMA uses (four chains, added
        // in a fixed order)
@@ -546,11 +566,7 @@ __global__ void __launch_bounds__(128) lin_apply_tc_kernel(
     zm[c] = zmar[i64(list_row) * kD + c];  // z^M, gathered by the indicator kernel
     ok = __syncthreads_and(wait_bounded(b_tma, 0, status, timeout));
     if (ok) {
-      for (int x = tid; x < BQ * 16; x += 128) {  // phi(Q) in place, padding rows zero
-        const int row = x >> 4, chunk = (x >> 3) & 1, u = x & 7;
-        uint4* p = reinterpret_cast<uint4*>(base + offQ + chunk * kQChunk + sw128(row, u));
-        *p = row < valid ? phi_unit(*p) : make_uint4(0u, 0u, 0u, 0u);
-      }
+      phi_tile<BQ>(base + offQ, kQChunk, valid, tid);  // phi(Q) in place, padding rows zero
       __syncthreads();
       for (int t = tid; t < BQ; t += 128) {  // normaliser from the rounded phi(q)
         float s = 0.f;
