@@ -51,7 +51,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum, the pipeline's own L2 contents, the timed step of
 # `bench.py --steps 1 --warmup 1`); absent = null.
 TRAFFIC_PER_LAUNCH = {
-    ("sla_1p3b", "attn_tc"): 506_990_336 + 136_226_048,
+    ("sla_1p3b", "attn_tc"): 507_496_960 + 135_902_208,
 }
 
 
