@@ -866,9 +866,13 @@ cudaError_t launch_select_rows(const float* in, int nrows, const Geom& g, int8_t
   a.tie_count = tie_count;
   const size_t per = select_per_warp_bytes(g.nkb, cdf);
   a.per_warp = static_cast<int>(per);
+  // Short rows (a warp's share at most 8 KB): CTAs of 2 warps, which the
+  // registers, not shared memory, then limit to ~20 resident warps per SM
+  // (measured faster than 1, 3, 6 or 8 at rows of 512 blocks).  Longer rows:
   // up to 8 warps (rows) per CTA, at most ~56 KB of shared memory each, so
-  // that several CTAs share an SM
-  const int warps = static_cast<int>(std::max<size_t>(1, std::min<size_t>(8, (56 * 1024) / per)));
+  // that several CTAs share an SM (measured best at rows of 1182 and 1920).
+  const int warps = per <= 8192 ? 2
+                                : static_cast<int>(std::max<size_t>(1, std::min<size_t>(8, (56 * 1024) / per)));
   const size_t smem = per * warps;
   const int grid = (nrows + warps - 1) / warps;
   cudaError_t e;
