@@ -308,18 +308,22 @@ def launches_per_step(wl, fused, bwd):
     """Kernels the library launches per step, from the entry points' code
     (checked against the ncu launch lists)."""
     # pool (Q and K in one launch), logits + selection per head group | plan
-    # (+ W to bf16, summaries, indicator, gather GEMM) | fused attention (or
-    # attention + combine)
-    n = 1 + 2 * mask_groups(wl) + (1 if fused else 0) + (4 if (fused and wl.frac_marg > 0) else 0) \
+    # (+ summaries, indicator, gather GEMM; W to bf16 rides in the indicator
+    # kernel unless B*H*Nqb < 16, when it takes a launch of its own) | fused
+    # attention (or attention + combine)
+    nqb = -(-wl.N // wl.block_q)
+    prep = 3 if wl.B * wl.H * nqb >= 16 else 4
+    n = 1 + 2 * mask_groups(wl) + (1 if fused else 0) + (prep if (fused and wl.frac_marg > 0) else 0) \
         + (1 if (not fused and wl.frac_marg > 0) else 0) + (1 if fused else 2)
     if bwd:
         lin = wl.frac_marg > 0
         n += 1  # column lists
         if fused and wl.d == 128:
             # Delta | 2 tile plans, dq (+ linear query side), dkdv (+ linear
-            # key side) | (W to bf16, summaries, indicator, gather of H^M,
-            # indicator + gather of dH, dW partials, dW sum)
-            n += 1 + 4 + (8 if lin else 0)
+            # key side) | (summaries, indicator, gather of H^M -- W to bf16
+            # as in the forward --, indicator + gather of dH, dW partials, dW
+            # sum)
+            n += 1 + 4 + ((prep + 4) if lin else 0)
         else:
             # Delta and g, dW partials | dq, dkdv (tcgen05: + 2 tile plans) |
             # (summaries, linear dq, linear dk dv) | dW reduction

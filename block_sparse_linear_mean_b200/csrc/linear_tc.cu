@@ -314,15 +314,25 @@ __global__ void __launch_bounds__(128) lin_summary_persist_kernel(
 //     CTA of 128 threads per query-block row.  Warp w sums the list entries
 //     e = w mod 4 (each lane four channels, one 16-byte load per entry, so a
 //     warp keeps several L2 reads in flight), and the four partial sums are
-//     added in a fixed order.
+//     added in a fixed order.  With w given, the first CTAs also write the
+//     projection W (fp32) as bf16 into wb for the fused epilogue (a launch
+//     of its own would cost more than the conversion).
 __global__ void __launch_bounds__(128) indicator_kernel(sla_block_lists rows,
                                                         uint16_t* __restrict__ ind,
                                                         const float* __restrict__ zsum,
                                                         float* __restrict__ zm, int nqb, int nkb,
-                                                        int ld) {
+                                                        int ld, const float* __restrict__ w,
+                                                        uint16_t* __restrict__ wb) {
   __shared__ int lst[256];
   __shared__ float4 part[4][32];
   const int row = blockIdx.x, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  constexpr int kWCtas = 16;  // CTAs sharing the conversion of W's kHElems entries
+  if (w && row < kWCtas) {
+    for (int i = row * 128 + tid; i < kHElems; i += kWCtas * 128) {
+      const __nv_bfloat16 b = __float2bfloat16_rn(w[i]);
+      wb[i] = *reinterpret_cast<const uint16_t*>(&b);
+    }
+  }
   const int bh = row / nqb;
   uint4* p = reinterpret_cast<uint4*>(ind + i64(row) * ld);
   for (int x = tid; x < ld / 8; x += blockDim.x) p[x] = make_uint4(0u, 0u, 0u, 0u);
@@ -738,7 +748,7 @@ cudaError_t launch_list_gather(const sla_block_lists& lists, int BH, int nrow, i
                                cudaStream_t s) {
   cudaError_t e;
   uint16_t* indp = static_cast<uint16_t*>(ind);
-  indicator_kernel<<<BH * nrow, 128, 0, s>>>(lists, indp, src_z, dst_z, nrow, ncol, ld);
+  indicator_kernel<<<BH * nrow, 128, 0, s>>>(lists, indp, src_z, dst_z, nrow, ncol, ld, nullptr, nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   CUtensorMap mA, mB, mC;
   const uint64_t bh = BH, nr = nrow, nc = ncol, l = ld;
@@ -816,8 +826,6 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
       return cudaErrorInvalidValue;
   }
   if (prepare) {
-  to_bf16_kernel<<<(kHElems + 255) / 256, 256, 0, s>>>(proj, wb, kHElems);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 1. summaries
   {
     const int debug_skip = debug_withhold(g, SLA_WITHHOLD_SUMMARIES) ? 1 : 0;
@@ -841,7 +849,13 @@ static cudaError_t lin_tc_impl(const void* q, const void* k, const void* v, cons
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 2. indicator + gather GEMM
-  indicator_kernel<<<g.BH * g.nqb, 128, 0, s>>>(rows, ind, zbuf, zmbuf, g.nqb, g.nkb, w.ld);
+  // (W to bf16 rides along in the first CTAs; 16 CTAs x 128 threads)
+  if (g.BH * g.nqb < 16) {
+    to_bf16_kernel<<<(kHElems + 255) / 256, 256, 0, s>>>(proj, wb, kHElems);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  indicator_kernel<<<g.BH * g.nqb, 128, 0, s>>>(rows, ind, zbuf, zmbuf, g.nqb, g.nkb, w.ld,
+                                                 g.BH * g.nqb >= 16 ? proj : nullptr, wb);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_gather(mA, mB, mC, w.ld, g.nqb, g.BH, status, g, s)) != cudaSuccess) return e;
   }  // prepare

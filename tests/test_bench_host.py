@@ -64,7 +64,7 @@ def test_tensor_peak_burst_under_a_second_sustained_above():
 
 def test_launch_counts_grow_with_the_head_groups():
     one = bench.launches_per_step(W["sla_1p3b"], True, False)
-    assert one == 1 + 2 + 1 + 4 + 1           # pool, logits + select, plan, linear, attention
+    assert one == 1 + 2 + 1 + 3 + 1           # pool, logits + select, plan, linear, attention
     assert bench.launches_per_step(W["long_clip"], True, False) == one + 2 * 13
     assert bench.launches_per_step(W["nabla_14b"], True, False) == 1 + 2 * 5 + 1 + 1
 
