@@ -81,7 +81,12 @@ static_assert(kMaxBlocks <= 8192, "plan entries hold 13-bit block indices");
 __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(sla_block_lists rows, int BH, int nqb,
                                                                int nkb, int nqt, int bq, int bk,
                                                                int32_t* __restrict__ cnt,
-                                                               uint32_t* __restrict__ tiles) {
+                                                               uint32_t* __restrict__ tiles,
+                                                               int32_t* __restrict__ zero_words,
+                                                               int nzero) {
+  // (the status words of the step's later kernels, zeroed here instead of by
+  // a memset of their own: no kernel before this one writes them)
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < nzero) zero_words[threadIdx.x] = 0;
   __shared__ uint32_t bits[kPlanWarps][2][kMaxBlocks / 32];
   const unsigned full = 0xffffffffu;
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -905,12 +910,13 @@ size_t attn_tc_scratch_bytes(const Geom& g) {
 }
 
 cudaError_t launch_attn_plan(const Geom& g, const sla_block_lists& rows, void* scratch,
-                             cudaStream_t s) {
+                             cudaStream_t s, int32_t* zero_words, int nzero) {
+  if (nzero > 32 * kPlanWarps) return cudaErrorInvalidValue;
   const int nqt = (g.N + kTileM - 1) / kTileM;
   const size_t ntiles = static_cast<size_t>(g.BH) * nqt;
   const PlanPtrs pp = plan_ptrs(g, scratch);
   plan_kernel<<<static_cast<unsigned>((ntiles + kPlanWarps - 1) / kPlanWarps), 32 * kPlanWarps, 0, s>>>(
-      rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, pp.cnt, pp.tiles);
+      rows, g.BH, g.nqb, g.nkb, nqt, g.bq, g.bk, pp.cnt, pp.tiles, zero_words, nzero);
   return cudaGetLastError();
 }
 
@@ -920,7 +926,7 @@ cudaError_t launch_tile_plan(const sla_block_lists& lists, int BH, int nrb, int 
   const size_t ntiles = static_cast<size_t>(BH) * nt;
   if (ntiles == 0) return cudaSuccess;
   plan_kernel<<<static_cast<unsigned>((ntiles + kPlanWarps - 1) / kPlanWarps), 32 * kPlanWarps, 0, s>>>(
-      lists, BH, nrb, ncb, nt, rb, cb, cnt, tiles);
+      lists, BH, nrb, ncb, nt, rb, cb, cnt, tiles, nullptr, 0);
   return cudaGetLastError();
 }
 

@@ -53,8 +53,11 @@ bool encode_f32_map(void* map, const void* ptr, int rank, const uint64_t* dims,
 // mask path
 // block means of Q (blocks of bq tokens) and K (blocks of bk) in one launch;
 // with qlo/klo given, split as hi (in qbar/kbar) + lo, both tf32
+// zero_words[0, nzero) (nzero <= 128) and *zero_one (if given) are zeroed by
+// the first CTA, for the step's later kernels.
 cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar,
-                        float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s);
+                        float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s,
+                        int32_t* zero_words = nullptr, int nzero = 0, int32_t* zero_one = nullptr);
 cudaError_t launch_logits(const float* qbar, const float* kbar, float* logits,
                           const Geom& g, cudaStream_t s);
 // the same logits on the tensor cores from the split means (logits_tc.cu)
@@ -151,8 +154,9 @@ struct LinInputs {
   const float* zm;         // fp32 z^M [B*H*Nqb, 128]
   const int32_t* marg_cnt; // marginal list counts [B*H*Nqb]
 };
+// zero_words[0, nzero) (nzero <= 128) are zeroed by the first CTA.
 cudaError_t launch_attn_plan(const Geom& g, const sla_block_lists& rows, void* scratch,
-                             cudaStream_t s);
+                             cudaStream_t s, int32_t* zero_words = nullptr, int nzero = 0);
 cudaError_t launch_attn_tc_fused(const void* q, const void* k, const void* v, const Geom& g,
                                  void* scratch, const AttnOutputs& o, const LinInputs* lin,
                                  int32_t* status, cudaStream_t s);

@@ -31,7 +31,16 @@ template <typename T>
 __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ xq, const T* __restrict__ xk,
                                                    float* __restrict__ outq, float* __restrict__ outk,
                                                    float* __restrict__ loq, float* __restrict__ lok,
-                                                   int N, int d, int bq, int bk) {
+                                                   int N, int d, int bq, int bk,
+                                                   int32_t* __restrict__ zero_words, int nzero,
+                                                   int32_t* __restrict__ zero_one) {
+  // words the later kernels of the step count or flag into (the status word
+  // block, the near-tie counter), zeroed here instead of by memsets of
+  // their own: no kernel before this one writes them
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
+    if (static_cast<int>(threadIdx.x) < nzero) zero_words[threadIdx.x] = 0;
+    if (threadIdx.x == 0 && zero_one) *zero_one = 0;
+  }
   constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
   constexpr int kU = 8;                // loads in flight per thread
   const bool isk = blockIdx.z == 1;
@@ -95,15 +104,17 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ xq, con
 }
 
 cudaError_t launch_pool(const void* q, const void* k, int dtype, float* qbar, float* kbar,
-                        float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s) {
+                        float* qlo, float* klo, int BH, int N, int d, int bq, int bk, cudaStream_t s,
+                        int32_t* zero_words, int nzero, int32_t* zero_one) {
+  if (nzero > 128) return cudaErrorInvalidValue;
   dim3 grid((N + min(bq, bk) - 1) / min(bq, bk), BH, 2);
   if (dtype == SLA_BF16)
     pool_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
                                                     static_cast<const __nv_bfloat16*>(k), qbar, kbar,
-                                                    qlo, klo, N, d, bq, bk);
+                                                    qlo, klo, N, d, bq, bk, zero_words, nzero, zero_one);
   else
     pool_kernel<float><<<grid, 128, 0, s>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                            qbar, kbar, qlo, klo, N, d, bq, bk);
+                                            qbar, kbar, qlo, klo, N, d, bq, bk, zero_words, nzero, zero_one);
   return cudaGetLastError();
 }
 

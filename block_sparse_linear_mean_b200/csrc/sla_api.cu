@@ -239,16 +239,19 @@ sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
   const MaskWs w = mask_ws(g);
   if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
   float* qbar = at<float>(ws, w.qbar);
   float* kbar = at<float>(ws, w.kbar);
   float* logits = at<float>(ws, w.logits);
-  if (tie_count) SLA_CUDA(cudaMemsetAsync(tie_count, 0, sizeof(int32_t), s));
+  // the status words and the near-tie counter are zeroed by the pooling
+  // kernel, the first of the step
+  int32_t* const zw = at<int32_t>(ws, 0);
+  constexpr int kZw = static_cast<int>(kStatusBytes / sizeof(int32_t));
   const size_t rowcols = size_t(g.nqb) * g.nkb;
   if (sla::logits_tc_supported(g)) {
     float* qlo = at<float>(ws, w.qlo);
     float* klo = at<float>(ws, w.klo);
-    SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, qlo, klo, g.BH, g.N, g.d, g.bq, g.bk, s));
+    SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, qlo, klo, g.BH, g.N, g.d, g.bq, g.bk, s, zw, kZw,
+                              tie_count));
     // logits and selection a group of heads at a time, through the slab
     const int G = mask_group_heads(g);
     for (int h0 = 0; h0 < g.BH; h0 += G) {
@@ -264,7 +267,7 @@ sla_status sla_build_mask(const sla_params* p, const void* q, const void* k,
     }
   } else {
     SLA_CUDA(sla::launch_pool(q, k, g.dtype, qbar, kbar, nullptr, nullptr, g.BH, g.N, g.d, g.bq, g.bk,
-                              s));
+                              s, zw, kZw, tie_count));
     const int G = mask_group_heads(g);
     for (int h0 = 0; h0 < g.BH; h0 += G) {
       Geom gg = g;
@@ -384,8 +387,13 @@ sla_status sla_forward_prepare(const sla_params* p, const void* k, const void* v
   const FwdWs w = fwd_ws(g);
   if (ws_bytes < w.total) return SLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
-  if (tc_attention(g)) SLA_CUDA(sla::launch_attn_plan(g, *rows, at<void>(ws, w.tc), s));
+  if (tc_attention(g)) {
+    // the plan kernel, the first of the step, zeroes the status words
+    SLA_CUDA(sla::launch_attn_plan(g, *rows, at<void>(ws, w.tc), s, at<int32_t>(ws, 0),
+                                   static_cast<int>(kStatusBytes / sizeof(int32_t))));
+  } else {
+    SLA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, s));
+  }
   if (has_linear_branch(g)) {
     if (sla::lin_tc_supported(g))
       SLA_CUDA(sla::launch_lin_tc_prepare(k, v, proj, *rows, g, at<void>(ws, w.lintc),
