@@ -296,11 +296,11 @@ RANGE_WORKLOADS = ("nabla_14b", "long_clip")
 
 def mask_groups(wl):
     """Head groups of the mask step: the logits of a group go through a slab
-    of at most 48 MB (the library's constant), one logits and one selection
+    of at most 64 MB (the library's constant), one logits and one selection
     launch per group."""
     nqb, nkb = math.ceil(wl.N / wl.block_q), math.ceil(wl.N / wl.block_k)
     bh = wl.B * wl.H
-    per_group = max(1, min(bh, (48 << 20) // (4 * nqb * nkb)))
+    per_group = max(1, min(bh, (64 << 20) // (4 * nqb * nkb)))
     return math.ceil(bh / per_group)
 
 
