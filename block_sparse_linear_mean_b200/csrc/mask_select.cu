@@ -19,7 +19,8 @@
 // histogram of counts (and, for the CDF rule, fixed-point masses) over equal
 // ranges of patterns spanning the row's scores; a scan over the
 // bins finds the bin holding each cut; the scores of that bin are compacted
-// and the cut value is resolved bit by bit among them; a last pass labels
+// and the cut value is read off a bitonic warp sort of them (up to 64, two
+// per lane), or resolved bit by bit among more; a last pass labels
 // the row in index order (equal scores fill the remaining slots by index),
 // writes the mask and the ascending block lists and counts near-ties.
 #include <float.h>
@@ -189,22 +190,45 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
 }
 
 // Bitonic sort of one key per lane across the warp, descending (the largest
-// at lane 0), carrying a payload: 15 compare-exchange steps over shuffles.
-// Blocks of k lanes alternate direction; the last stage (k = 32) runs
-// descending over the whole warp.
-__device__ __forceinline__ void warp_sort_desc(uint32_t& x, unsigned long long& pay, int lane) {
+// at lane 0): 15 compare-exchange steps over shuffles.  Blocks of k lanes
+// alternate direction; the last stage (k = 32) runs descending over the
+// whole warp.  Only keys move: a candidate's mass is a function of its key,
+// recomputed after the sort.
+__device__ __forceinline__ uint32_t warp_sort_desc(uint32_t x, int lane) {
 #pragma unroll
   for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1) {
       const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
-      const unsigned long long py = __shfl_xor_sync(0xffffffffu, pay, j);
-      const bool desc = (lane & k) == 0;
-      const bool low = (lane & j) == 0;
-      const bool take_max = low == desc;
-      const bool swap = take_max ? (y > x) : (y < x);
-      if (swap) { x = y; pay = py; }
+      const bool take_max = ((lane & j) == 0) == ((lane & k) == 0);
+      x = take_max ? max(x, y) : min(x, y);
     }
+  }
+  return x;
+}
+
+// The same over 64 keys, two per lane: key r of lane l is element 2l + r,
+// so the sorted order runs lane 0 (x0 >= x1), lane 1, ...  An element's
+// block direction (element & k) is lane & k/2; at distances of 2 and more
+// lane l meets lane l ^ j/2 (each key with its namesake), at distance 1 a
+// lane orders its own two keys: 15 exchange steps over shuffles, 6 in
+// registers.
+__device__ __forceinline__ void warp_sort64_desc(uint32_t& x0, uint32_t& x1, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+    const bool desc = (lane & (k >> 1)) == 0;
+#pragma unroll
+    for (int j = k >> 1; j >= 2; j >>= 1) {
+      const int lj = j >> 1;
+      const uint32_t y0 = __shfl_xor_sync(0xffffffffu, x0, lj);
+      const uint32_t y1 = __shfl_xor_sync(0xffffffffu, x1, lj);
+      const bool take_max = ((lane & lj) == 0) == desc;
+      x0 = take_max ? max(x0, y0) : min(x0, y0);
+      x1 = take_max ? max(x1, y1) : min(x1, y1);
+    }
+    const uint32_t hi = max(x0, x1), lo = min(x0, x1);
+    x0 = desc ? hi : lo;
+    x1 = desc ? lo : hi;
   }
 }
 
@@ -214,28 +238,39 @@ __device__ __forceinline__ void warp_sort_desc(uint32_t& x, unsigned long long& 
 // level with every real one, which leaves the value at rank need - 1 as it is.
 __device__ __forceinline__ void rank_small(uint32_t c, bool have, int need, int lane, uint32_t& v,
                                            int& above, int& eq) {
-  uint32_t key = have ? c : 0u;
-  unsigned long long none = 0;
-  warp_sort_desc(key, none, lane);
+  const uint32_t key = warp_sort_desc(have ? c : 0u, lane);
   v = __shfl_sync(0xffffffffu, key, need - 1);
   above = __popc(__ballot_sync(0xffffffffu, have && c > v));
   eq = __popc(__ballot_sync(0xffffffffu, have && c == v));
 }
 
+// rank_small over 32 < n <= 64 candidates, two per lane (c0 always held, c1
+// where h1): rank need - 1 is element need - 1 of the sorted order.
+__device__ __forceinline__ void rank_pair(uint32_t c0, uint32_t c1, bool h1, int need, int lane,
+                                          uint32_t& v, int& above, int& eq) {
+  uint32_t k0 = c0, k1 = h1 ? c1 : 0u;
+  warp_sort64_desc(k0, k1, lane);
+  const int p = need - 1;
+  const uint32_t s0 = __shfl_sync(0xffffffffu, k0, p >> 1);
+  const uint32_t s1 = __shfl_sync(0xffffffffu, k1, p >> 1);
+  v = (p & 1) ? s1 : s0;
+  above = __popc(__ballot_sync(0xffffffffu, c0 > v)) + __popc(__ballot_sync(0xffffffffu, h1 && c1 > v));
+  eq = __popc(__ballot_sync(0xffffffffu, c0 == v)) + __popc(__ballot_sync(0xffffffffu, h1 && c1 == v));
+}
+
 // CDF cut among n <= 32 candidates held one per lane: the candidate v at
 // which lo + (mass of the candidates <= v) first reaches thr, the mass under
 // it (`below`, lo included), and the candidates above and equal to it.
-// Sorted descending with their masses, the suffix sums S_L (lane L and
-// every lane after it) decrease with L; v is the key at the last lane with
+// Sorted descending, the suffix sums S_L of the masses (lane L and every
+// lane after it) decrease with L; v is the key at the last lane with
 // lo + S_L >= thr (a lane of v's group: the group's first lane holds the
 // mass of everything <= v, the lane after the group only what is below v).
 __device__ __forceinline__ void mass_small(uint32_t c, bool have, unsigned long long lo,
                                            uint64_t thr, int lane, uint32_t& v,
                                            unsigned long long& below, int& above, int& eq) {
   const unsigned long long fx = have ? to_fixed(c) : 0ull;
-  uint32_t key = have ? c : 0u;
-  unsigned long long m = fx;
-  warp_sort_desc(key, m, lane);
+  const uint32_t key = warp_sort_desc(have ? c : 0u, lane);
+  const unsigned long long m = to_fixed(key);  // (0 for the padding)
   unsigned long long suf = m;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -251,6 +286,39 @@ __device__ __forceinline__ void mass_small(uint32_t c, bool have, unsigned long 
   below = lo + under;
   above = __popc(__ballot_sync(0xffffffffu, have && c > v));
   eq = __popc(__ballot_sync(0xffffffffu, have && c == v));
+}
+
+// mass_small over 32 < n <= 64 candidates, two per lane (c0 always held, c1
+// where h1).  In the sorted order lane l holds elements 2l and 2l + 1; with
+// U_l the suffix sum of the lanes' pair masses, S(2l) = U_l and
+// S(2l + 1) = U_l - m(2l), and v is the key at the last element whose
+// lo + S reaches thr.
+__device__ __forceinline__ void mass_pair(uint32_t c0, uint32_t c1, bool h1, unsigned long long lo,
+                                          uint64_t thr, int lane, uint32_t& v,
+                                          unsigned long long& below, int& above, int& eq) {
+  uint32_t k0 = c0, k1 = h1 ? c1 : 0u;
+  warp_sort64_desc(k0, k1, lane);
+  const unsigned long long m0 = to_fixed(k0), m1 = to_fixed(k1);
+  unsigned long long suf = m0 + m1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  const unsigned w0 = __ballot_sync(0xffffffffu, lo + suf >= thr && m0 > 0);
+  const unsigned w1 = __ballot_sync(0xffffffffu, lo + (suf - m0) >= thr && m1 > 0);
+  const int l0 = w0 ? 31 - __clz(w0) : -1, l1 = w1 ? 31 - __clz(w1) : -1;
+  const bool odd = l1 >= 0 && 2 * l1 + 1 > 2 * l0;
+  const int src = odd ? l1 : max(l0, 0);
+  const uint32_t s0 = __shfl_sync(0xffffffffu, k0, src);
+  const uint32_t s1 = __shfl_sync(0xffffffffu, k1, src);
+  v = odd ? s1 : s0;
+  unsigned long long under = (c0 < v ? to_fixed(c0) : 0ull) + ((h1 && c1 < v) ? to_fixed(c1) : 0ull);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) under += __shfl_xor_sync(0xffffffffu, under, o);
+  below = lo + under;
+  above = __popc(__ballot_sync(0xffffffffu, c0 > v)) + __popc(__ballot_sync(0xffffffffu, h1 && c1 > v));
+  eq = __popc(__ballot_sync(0xffffffffu, c0 == v)) + __popc(__ballot_sync(0xffffffffu, h1 && c1 == v));
 }
 
 // Shared memory of one warp (byte offsets; 16-byte aligned pieces).
@@ -475,6 +543,8 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
       rank_in_bin(b, need, v, above, eq);
     } else if (n <= 32) {
       rank_small(lane < n ? cl[lane] : 0u, lane < n, need, lane, v, above, eq);
+    } else if (n <= 64) {
+      rank_pair(cl[lane], lane + 32 < n ? cl[lane + 32] : 0u, lane + 32 < n, need, lane, v, above, eq);
     } else {
       v = rank_among(cl, n, need, lane);
       above = count_greater(cl, n, v, lane);
@@ -582,6 +652,9 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
         int above, g;
         if (fit && n <= 32) {
           mass_small(lane < n ? cand[lane] : 0u, lane < n, lo, a.thr_fx, lane, v, below, above, g);
+        } else if (fit && n <= 64) {
+          mass_pair(cand[lane], lane + 32 < n ? cand[lane + 32] : 0u, lane + 32 < n, lo, a.thr_fx, lane,
+                    v, below, above, g);
         } else {
           // bit by bit: the largest t whose mass below it stays under thr
           uint32_t t = 0;
