@@ -614,13 +614,34 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
       bin_from_bottom(hcnt, hmass, static_cast<uint32_t>(a.thr_fx >> 38), lane, b, lo, ab, found);
       if (!found) b = 255;
       found = false;
+      // (the first pass also collects bin b's scores as the cut's candidates,
+      // the gather of step 4; the pass is usually the only one)
+      int gathered = -1;
       for (int it = 0; it <= kBins; ++it) {
         unsigned long long s_lo = 0, s_b = 0;
-        for (int j = lane; j < nkb; j += 32) {
-          const uint32_t x = pb[j];
-          const int bx = bin_of(x, base, shift);
-          if (bx < b) s_lo += to_fixed(x);
-          else if (bx == b) s_b += to_fixed(x);
+        const bool take = it == 0;
+        for (int g = lane; g < G; g += 32) {
+          const uint32_t bb = bins[g];
+          const uint4 v4 = pb4[g];
+          const uint32_t v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (4 * g + k >= nkb) continue;
+            const int bx = static_cast<int>((bb >> (8 * k)) & 255u);
+            if (bx < b) {
+              s_lo += to_fixed(v[k]);
+            } else if (bx == b) {
+              s_b += to_fixed(v[k]);
+              if (take) {
+                const uint32_t sl = atomicAdd(&ctr[0], 1u);
+                if (sl < kCand) cand[sl] = v[k];
+              }
+            }
+          }
+        }
+        if (take) {
+          __syncwarp();
+          gathered = b;
         }
         s_lo = warp_sum_u64(s_lo);
         s_b = warp_sum_u64(s_b);
@@ -645,7 +666,13 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
         uint32_t nab = 0;
         for (int i = lane; i < kBins; i += 32) nab += i > b ? hcnt[i] : 0u;
         ab = static_cast<int>(__reduce_add_sync(full, nab));
-        const bool fit = gather(b, -1);
+        bool fit = ctr[0] <= static_cast<uint32_t>(kCand);
+        if (gathered != b) {  // the cut moved to another bin: collect that one's
+          __syncwarp();
+          if (lane < 2) ctr[lane] = 0u;
+          __syncwarp();
+          fit = gather(b, -1);
+        }
         const int n = static_cast<int>(min(ctr[0], static_cast<uint32_t>(kCand)));
         uint32_t v;
         unsigned long long below;
