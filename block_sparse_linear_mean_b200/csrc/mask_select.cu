@@ -345,7 +345,9 @@ __device__ __forceinline__ bool has_byte(uint32_t x, uint32_t b) {
   return ((y - 0x01010101u) & ~y & 0x80808080u) != 0;
 }
 
-template <bool CDF>
+// MARG = false compiles the kernel without the marginal cut (for rules
+// that keep no marginal blocks, n_m = 0: the usual NABLA use).
+template <bool CDF, bool MARG>
 __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restrict__ in,
                                                           SelectArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -559,7 +561,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
   int c = 0;
   if (!CDF) {
     c = a.n_c;
-    const int nm = min(a.n_m, nkb - c);
+    const int nm = MARG ? min(a.n_m, nkb - c) : 0;
     int bc = -1, ab_c = 0, bm = -1, ab_m = 0;
     if (c > 0) bin_from_top(hcnt, c, lane, bc, ab_c);
     if (nm > 0) bin_from_top(hcnt, c + nm, lane, bm, ab_m);
@@ -769,7 +771,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const float* __restric
         }
       }
     }
-    const int nm = min(a.n_m, nkb - c);
+    const int nm = MARG ? min(a.n_m, nkb - c) : 0;
     if (nm > 0) {
       int bm = 0, ab_m = 0;
       bin_from_top(hcnt, c + nm, lane, bm, ab_m);
@@ -975,18 +977,17 @@ cudaError_t launch_select_rows(const float* in, int nrows, const Geom& g, int8_t
                                 : static_cast<int>(std::max<size_t>(1, std::min<size_t>(8, (56 * 1024) / per)));
   const size_t smem = per * warps;
   const int grid = (nrows + warps - 1) / warps;
+  auto launch = [&](auto kern) -> cudaError_t {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 32 * warps, smem, s>>>(in, a);
+    return cudaSuccess;
+  };
   cudaError_t e;
-  if (cdf) {
-    if ((e = cudaFuncSetAttribute(select_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(smem))) != cudaSuccess)
-      return e;
-    select_rows_kernel<true><<<grid, 32 * warps, smem, s>>>(in, a);
-  } else {
-    if ((e = cudaFuncSetAttribute(select_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(smem))) != cudaSuccess)
-      return e;
-    select_rows_kernel<false><<<grid, 32 * warps, smem, s>>>(in, a);
-  }
+  if (cdf) e = g.n_m > 0 ? launch(select_rows_kernel<true, true>) : launch(select_rows_kernel<true, false>);
+  else e = launch(select_rows_kernel<false, true>);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
