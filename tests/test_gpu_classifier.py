@@ -100,3 +100,32 @@ def test_classifier_at_the_longest_rows(kind, mode, fc, fm, thr):
     exp = expected_rows(mask[None, None])
     assert [lists[0][r] for r in sample] == exp[0]
     assert [lists[1][r] for r in sample] == exp[1]
+
+
+@pytest.mark.parametrize("n_small", [40, 300])
+@pytest.mark.parametrize("fm", [0.0, 0.05])
+def test_cdf_cut_moved_to_a_lower_bin_by_the_exact_sums(n_small, fm):
+    # n_small equal small scores whose 2^-24-unit truncation (the histogram's
+    # approximate masses) loses almost a unit each, and 60 scores of 2^-7:
+    # thr is exactly the small scores' total, so the approximate masses put
+    # the cut in the large scores' bin and the exact fixed-point sums move it
+    # down to the small scores' bin, whose scores are then collected anew
+    # (40: a cut among 33-64 candidates; 300: more than the 256 slots, the
+    # search over the whole row).  The one small score whose tail sum equals
+    # thr exactly is kept, and every row is a near-tie row.
+    a = np.float32((2046 + 1014 / 1024) * 2.0 ** -24)
+    assert float(a) == (2046 + 1014 / 1024) * 2.0 ** -24
+    thr = n_small * float(a)  # dyadic: exact in binary64 and in 2^-62 fixed point
+    nkb = n_small + 60
+    rng = np.random.default_rng(n_small)
+    row = np.concatenate([np.full(n_small, a, np.float32), np.full(60, np.float32(2.0 ** -7))])
+    s32 = np.stack([rng.permutation(row) for _ in range(nkb)]).astype(np.float32)
+    wl, p = _params(nkb, nkb, "cdf", 0.0, fm, thr)
+    got = sla.classify_scores(p, torch.from_numpy(s32.reshape(1, 1, nkb, nkb)).cuda())
+    torch.cuda.synchronize()
+    mask = got["mask"].cpu().numpy()[0, 0]
+    ref, margins = orc.classify(s32.astype(np.float64), "cdf", 0.0, fm, thr)
+    assert ((ref == 2).sum(axis=1) == 61).all()
+    np.testing.assert_array_equal(mask, ref)
+    assert lists_from_gpu(got["rows"], nkb, nkb) == expected_rows(mask[None, None])
+    assert int(got["ties"].item()) == int((margins <= 1e-5).sum()) == nkb
